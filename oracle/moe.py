@@ -1,0 +1,88 @@
+"""MoE expert-FFN layer of the QUADS rollout engine, per token -- TEST
+INFRASTRUCTURE ONLY (see oracle/__init__.py).
+
+The layer (QUADS pages: gist.science/it sections 1 and 4 -- a routed MoE whose
+expert GEMMs run as native W4A4 NVFP4 products; section 2.2 B -- Residual
+Activation Compensation on the activations entering each GEMM):
+
+    idx, g   = top-k_r routing of the router logits, softmax over the k_r
+    Xq       = NVFP4(X)                       (one s_t over all tokens)
+    S_x      = top-k channels of X's residual score
+    y13[t,j] = Xhat[t] W13q_e^T + s_x rho_x[t] W13q_e[:, S_x]^T,  e = idx[t,j]
+    h[t,j]   = bf16(silu(y13[:, :I]) * y13[:, I:])
+    Hq       = NVFP4(h over all routed rows)  (one s_t, one S_h)
+    y2[t,j]  = Hhat[t,j] W2q_e^T + s_h rho_h[t,j] W2q_e[:, S_h]^T
+    Y[t]     = sum_j g[t,j] y2[t,j]
+
+Weights are quantized per expert tensor, each with its own s_t.  Routed rows
+are kept in (token, slot) order, row t*k_r + j; the order is irrelevant to
+every quantity above except the binary64 summation order of the h scores.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import (quantize, select_topk, channel_score, rac_residual, route,
+               w4a4_rac_matmul, swiglu, f32_to_bf16, bf16_to_f32)
+
+
+def quantize_weights(w: np.ndarray):
+    """Per-expert NVFP4 weights: list of oracle.Quantized, one per expert,
+    each with its own tensor scale."""
+    return [quantize(w[e]) for e in range(w.shape[0])]
+
+
+def gate_up(xq, rho_x, S_x, idx, w13q, inter):
+    """y13 for every routed row (t, j) and h = swiglu(y13).
+    Returns (h_f64 [T*kr, I], h_bf16 [T*kr, I])."""
+    T, kr = idx.shape
+    h = np.zeros((T * kr, inter), np.float64)
+    rows_t = np.repeat(np.arange(T), kr)
+    experts = idx.reshape(-1)
+    for e in np.unique(experts):
+        rows = np.nonzero(experts == e)[0]
+        toks = rows_t[rows]
+        y = w4a4_rac_matmul(xq.xhat[toks], xq.s_t, None if rho_x is None else rho_x[toks],
+                            S_x, w13q[e].xhat)
+        h[rows] = swiglu(y, inter)
+    return h, f32_to_bf16(h.astype(np.float32))
+
+
+def down(h_bf16, idx, gate, w2q, k_h, row_valid=None):
+    """Quantize the routed h rows as one tensor, select S_h, run the down GEMM
+    with RAC and combine with the router weights.
+    Returns dict(Y [T, H] f64, hq, S_h, rho_h, y2 [T*kr, H])."""
+    T, kr = idx.shape
+    hq = quantize(h_bf16)
+    S_h = select_topk(channel_score(hq.resid, row_valid), k_h)
+    rho_h = rac_residual(hq.resid, hq.s_t, S_h)
+    H = w2q[0].xhat.shape[0]
+    y2 = np.zeros((T * kr, H), np.float64)
+    experts = idx.reshape(-1)
+    for e in np.unique(experts):
+        rows = np.nonzero(experts == e)[0]
+        y2[rows] = w4a4_rac_matmul(hq.xhat[rows], hq.s_t, rho_h[rows], S_h, w2q[e].xhat)
+    Y = (y2.reshape(T, kr, H) * gate[:, :, None]).sum(axis=1)
+    return dict(Y=Y, hq=hq, S_h=S_h, rho_h=rho_h, y2=y2)
+
+
+def layer(x, logits, w13q, w2q, kr, k_x, k_h):
+    """Full layer from bf16 X and router logits; weights already quantized."""
+    idx, gate = route(logits, kr)
+    xq = quantize(x)
+    S_x = select_topk(channel_score(xq.resid), k_x)
+    rho_x = rac_residual(xq.resid, xq.s_t, S_x)
+    inter = w13q[0].xhat.shape[0] // 2
+    h64, hb = gate_up(xq, rho_x, S_x, idx, w13q, inter)
+    out = down(hb, idx, gate, w2q, k_h)
+    out.update(idx=idx, gate=gate, xq=xq, S_x=S_x, rho_x=rho_x, h64=h64, h_bf16=hb)
+    return out
+
+
+def tokens_sample(x, logits, tokens):
+    """Restrict a layer's token inputs to a subset of tokens (used for the
+    large workloads, where the oracle runs on a sample)."""
+    return x[tokens], logits[tokens]
+
+
+__all__ = ["quantize_weights", "gate_up", "down", "layer", "tokens_sample", "bf16_to_f32"]
