@@ -1,0 +1,395 @@
+"""Benchmark of the QUADS rollout MoE layer hot path on B200.
+
+One step = one forward of the large MoE layer (T=16384 tokens, H=4096,
+I=1536, E=128 experts, top-8 routing with per-expert logit skew, RAC k=128
+per GEMM): routing, NVFP4 quantization of X with residual scores, top-k
+channel selection and RAC residuals, RAC weight gather, the grouped W4A4+RAC
+gate/up GEMM with SwiGLU, quantization of h, gather, the grouped W4A4+RAC down
+GEMM with router-weighted combine.  Weights are NVFP4 before timing (the
+rollout engine holds quantized weights).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs an independent replica on its own batch (weak scaling, no collective on
+the data path); time is the max over ranks.
+
+Prints one JSON line (rank 0).  value = whole-job algorithmic TFLOP/s of the
+layer (FP4 + RAC FLOPs of both GEMMs, padding not counted) over the device
+time of the K timed steps.  The reference arm (--impl reference) times the CPU
+oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "moe_t16384_e128"
+METRIC = "W4A4+RAC grouped MoE GEMM TFLOPS and % FP4 peak; quantize GB/s and % HBM"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP4_PER_BF16 = 4.0          # nominal dense FP4 : BF16 tensor-core ratio (9 : 2.25 PFLOP/s)
+QUANT_BYTES_PER_ELEM = 2.5625   # 2 B bf16 read + 0.5 B codes + 1/16 B scale written
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), source="measured")
+    except Exception:
+        return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sus=1400.0, source="fallback")
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend: str):
+    import datetime
+    import torch.distributed as dist
+    ws, rank, _ = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return ws, rank
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, enabled: bool = True):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"nvfp4_clocks_{os.getpid()}.csv")
+        self.gpu = gpu_index
+        if enabled:
+            try:
+                self.f = open(self.path, "w")
+                self.proc = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.QUERY}",
+                                              "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                             stderr=subprocess.DEVNULL)
+            except Exception:
+                self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [s.strip() for s in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    mx = float(p[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.remove(self.path)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 300] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    from quantization_nvfp4_quantize_b200 import workloads as wl, api
+    from quantization_nvfp4_quantize_b200.moe import MoELayerW4A4
+
+    ws, rank = init_dist("nccl" if torch.cuda.is_available() else "gloo")
+    _, _, local = dist_env()
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = wl.CONFIGS[args.workload]
+    seed = args.seed + rank                      # independent replica per rank
+    x = wl.activations(cfg, seed, device=dev)
+    logits = wl.router_logits(cfg, seed, device=dev)
+    w13, w2 = wl.weights(cfg, seed, device=dev)
+    layer = MoELayerW4A4(w13, w2, cfg.tokens, cfg.topk, cfg.rac_k)
+    del w13, w2
+    torch.cuda.empty_cache()
+    fl = wl.flops(cfg)
+    step_flops = fl["fp4"] + fl["rac"]
+    stream = torch.cuda.current_stream(dev)
+
+    # per-kernel timing hooks around the two GEMMs and the two quantize calls
+    ev = {"gemm": [], "quant": []}
+    orig_gemm, orig_quant = api.grouped_gemm, api.quantize
+
+    def timed(kind, fn):
+        def wrap(*a, **k):
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            out = fn(*a, **k)
+            e.record(stream)
+            ev[kind].append((s, e, a, k))
+            return out
+        return wrap
+
+    for _ in range(args.warmup):
+        layer.forward(x, logits)
+    torch.cuda.synchronize()
+    barrier()
+
+    api.grouped_gemm, api.quantize = timed("gemm", orig_gemm), timed("quant", orig_quant)
+    import quantization_nvfp4_quantize_b200.moe as moe_mod
+    moe_mod.api = api
+    clocks = ClockSampler(local, enabled=not args.no_clocks)
+    torch.cuda.synchronize()
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        layer.forward(x, logits)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    api.grouped_gemm, api.quantize = orig_gemm, orig_quant
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms, dev)
+
+    gemm_ms = sum(s.elapsed_time(e) for s, e, _, _ in ev["gemm"])
+    quant_ms = sum(s.elapsed_time(e) for s, e, _, _ in ev["quant"])
+    n_gemm = len(ev["gemm"])
+    # algorithmic work per step
+    M = cfg.tokens * cfg.topk
+    quant_elems = cfg.tokens * cfg.hidden + M * cfg.inter
+    p = peaks()
+    fp4_peak = p["bf16_sus"] * FP4_PER_BF16
+    gemm_fp4_tflops = fl["fp4"] * args.steps / (gemm_ms * 1e-3) / 1e12
+    gemm_all_tflops = step_flops * args.steps / (gemm_ms * 1e-3) / 1e12
+    quant_gbs = quant_elems * QUANT_BYTES_PER_ELEM * args.steps / (quant_ms * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(layer, x, logits, args, dev)
+    n_launch_per_step = 16
+    out = {
+        "metric": METRIC,
+        "value": round(step_flops * args.steps * ws / (ms_max * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e2m1+e4m3 (fp32 accum), bf16 RAC", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: T={cfg.tokens} H={cfg.hidden} I={cfg.inter} E={cfg.experts} "
+                               f"top-{cfg.topk} RAC k={cfg.rac_k}",
+                   "l2": "inputs larger than L2 (NVFP4 weights 1.36 GB)", "parallelism": f"replicas x{ws}"},
+        "roofline": {"bound": "tensor", "kernel": "k_moe_gemm",
+                     "achieved": round(gemm_fp4_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_fp4_tflops / fp4_peak, 4), "traffic": None,
+                     "peak_source": f"{p['source']} bf16 sustained x{FP4_PER_BF16:g} (nominal FP4:BF16)",
+                     "achieved_incl_rac": round(gemm_all_tflops, 1),
+                     "gemm_ms_per_step": round(gemm_ms / args.steps, 4), "launches_per_step": n_gemm // args.steps},
+        "quantize": {"gbs": round(quant_gbs, 1), "peak_gbs": p["hbm"], "frac": round(quant_gbs / p["hbm"], 4),
+                     "ms_per_step": round(quant_ms / args.steps, 4),
+                     "bytes_per_elem": QUANT_BYTES_PER_ELEM, "elems_per_step": quant_elems},
+        "e2e": e2e,
+        "gpu_launches": n_launch_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1:
+        out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=8)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return out
+
+
+def run_e2e(layer, x, logits, args, dev):
+    """Same metric through the public API with host buffers: every step copies
+    X and the router logits from pinned host memory and Y back."""
+    import torch
+    xh = x.cpu().pin_memory()
+    lh = logits.cpu().pin_memory()
+    yh = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
+    xd = torch.empty_like(x)
+    ld = torch.empty_like(logits)
+    stream = torch.cuda.current_stream(dev)
+    steps = max(1, args.steps // 2)
+    for _ in range(2):
+        xd.copy_(xh, non_blocking=True)
+        ld.copy_(lh, non_blocking=True)
+        yh.copy_(layer.forward(xd, ld), non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        xd.copy_(xh, non_blocking=True)
+        ld.copy_(lh, non_blocking=True)
+        yh.copy_(layer.forward(xd, ld), non_blocking=True)
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e), dev)
+    from quantization_nvfp4_quantize_b200 import workloads as wl
+    cfg = wl.CONFIGS[args.workload]
+    fl = wl.flops(cfg)
+    ws = dist_env()[0]
+    return {"value": round((fl["fp4"] + fl["rac"]) * steps * ws / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": xh.numel() * xh.element_size() + lh.numel() * lh.element_size(),
+            "d2h_bytes_per_step": yh.numel() * yh.element_size()}
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(cfg, seed=0, n_experts=8):
+    """The oracle, as it stands, on a bounded sample of the workload: every
+    routed row of the first `n_experts` experts (their tokens' X rows are
+    quantized, scored and selected, then both W4A4+RAC products, SwiGLU and
+    the h quantization run on those rows).  Weight quantization is done
+    before timing, as on the GPU.  Returns TFLOP/s of the sample."""
+    import numpy as np
+    import torch
+    import oracle
+    from quantization_nvfp4_quantize_b200 import workloads as wl
+
+    x = wl.activations(cfg, seed)
+    logits = wl.router_logits(cfg, seed)
+    xn = x.view(torch.int16).numpy().view(np.uint16)
+    idx, gate = oracle.route(logits.numpy(), cfg.topk)
+    g = torch.Generator().manual_seed(1234)
+    E_s = n_experts
+    w13 = [(torch.randn(2 * cfg.inter, cfg.hidden, generator=g) * 0.02).to(torch.bfloat16) for _ in range(E_s)]
+    w2 = [(torch.randn(cfg.hidden, cfg.inter, generator=g) * 0.02).to(torch.bfloat16) for _ in range(E_s)]
+    w13q = [oracle.quantize(w.view(torch.int16).numpy().view(np.uint16)).xhat for w in w13]
+    w2q = [oracle.quantize(w.view(torch.int16).numpy().view(np.uint16)).xhat for w in w2]
+    rows = [(t, j) for e in range(E_s) for t, j in zip(*np.nonzero(idx == e))]
+    toks = np.array(sorted({t for t, _ in rows}))
+    k = cfg.rac_k
+    t0 = time.perf_counter()
+    qx = oracle.quantize(xn[toks])
+    S_x = oracle.select_topk(oracle.channel_score(qx.resid), k)
+    rho_x = oracle.rac_residual(qx.resid, qx.s_t, S_x)
+    pos = {t: i for i, t in enumerate(toks)}
+    h = []
+    for e in range(E_s):
+        tt = np.array([pos[t] for t, j in rows if idx[t, j] == e], dtype=np.int64)
+        y = oracle.w4a4_rac_matmul(qx.xhat[tt], qx.s_t, rho_x[tt], S_x, w13q[e])
+        h.append(oracle.f32_to_bf16(oracle.swiglu(y, cfg.inter).astype(np.float32)))
+    hb = np.concatenate(h)
+    qh = oracle.quantize(hb)
+    S_h = oracle.select_topk(oracle.channel_score(qh.resid), k)
+    rho_h = oracle.rac_residual(qh.resid, qh.s_t, S_h)
+    start = 0
+    for e in range(E_s):
+        n = h[e].shape[0]
+        oracle.w4a4_rac_matmul(qh.xhat[start:start + n], qh.s_t, rho_h[start:start + n], S_h, w2q[e])
+        start += n
+    dt = time.perf_counter() - t0
+    M = len(rows)
+    flops = 2.0 * M * (2 * cfg.inter * cfg.hidden + cfg.hidden * cfg.inter) + \
+        2.0 * M * (2 * cfg.inter + cfg.hidden) * k
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"all {M} routed rows of experts 0..{E_s - 1} ({len(toks)} tokens) of {cfg.name}; "
+                      f"weights of those experts quantized before timing"}
+
+
+def run_reference(args):
+    """--impl reference: the oracle as it stands on the host cores, each step a
+    bounded sample (the routed rows of 2 experts) of the same workload."""
+    ws, rank = init_dist("gloo")
+    if rank != 0:
+        return None
+    from quantization_nvfp4_quantize_b200 import workloads as wl
+    cfg = wl.CONFIGS[args.workload]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(cfg, seed=args.seed, n_experts=2)
+        if i >= args.warmup:
+            vals.append(r)
+    tot_s = sum(v["seconds"] for v in vals)
+    value = statistics.mean(v["value"] for v in vals)
+    out = {"impl": "reference", "metric": METRIC,
+           "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / max(1, len(vals)), 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+           "data": "synthetic",
+           "config": {"workload": f"{cfg.name}: T={cfg.tokens} H={cfg.hidden} I={cfg.inter} E={cfg.experts} "
+                                  f"top-{cfg.topk} RAC k={cfg.rac_k}"},
+           "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": vals[0]["cores"],
+                            "kind": "oracle", "sample": vals[0]["sample"]},
+           "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return out
+
+
+def main():
+    args = parse()
+    try:
+        if args.impl == "reference":
+            run_reference(args)
+        else:
+            run_ours(args)
+    finally:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

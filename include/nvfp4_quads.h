@@ -1,0 +1,267 @@
+/*
+ * nvfp4_quads.h -- C ABI of the B200 (sm_100a) QUADS rollout hot path:
+ * NVFP4 online activation quantization with residual channel scoring,
+ * top-k high-residual channel selection, the token-permuted grouped W4A4 MoE
+ * expert GEMM with Residual Activation Compensation (RAC), and the
+ * trainer-side weight quantize-dequantize (QDQ, asymmetric W4A16 QAT).
+ *
+ * Sources (the QUADS pages; page, section):
+ *   gist.science/it, section 1      native W4A4 FP4 GEMMs; coarse E2M1 grid
+ *   shd-paper.top, English abstract NVFP4 = fine-grained scaling + native W4A4
+ *                                   GEMMs; activations are quantized online
+ *   gist.science/it, section 2.1    activations recomputed online are the
+ *                                   dominant error source
+ *   gist.science/it, section 2.2 A  trainer fake-quantizes weights (W4A16)
+ *   gist.science/it, section 2.2 B  RAC: top-k high-residual channels by a
+ *                                   binary channel mask, correction added back
+ *                                   to the quantized output, bulk stays on the
+ *                                   native W4A4 GEMM
+ *
+ * Conventions (every entry point):
+ *   - Pointers named *_dev are device pointers; the caller allocates and owns
+ *     every buffer.  The library allocates nothing: scratch memory is a
+ *     caller-provided workspace whose size the matching *_workspace_size
+ *     function returns.  Workspaces need no initialization.
+ *   - Calls are asynchronous on the given cudaStream_t (passed as void*;
+ *     NULL = legacy default stream) and return after enqueueing.
+ *   - Argument errors are detected synchronously and returned without
+ *     enqueueing anything; nvfp4_last_error_string() describes the last one.
+ *     NVFP4_ERR_CUDA reports a failed launch or runtime call.
+ *   - Device-side bounded waits that run out (a deadlock would otherwise
+ *     hang the GPU) write NVFP4_ERR_TIMEOUT into *dev_status when dev_status
+ *     is non-NULL; the kernel then drains its copies, frees its tensor memory
+ *     and returns.  Read it with nvfp4_read_status().
+ *   - Device pointers must be 16-byte aligned.  Tensors are dense row-major.
+ *   - Inputs must be finite; a tensor's max |x| must be 0 or >= 2^-90.
+ *
+ * Data formats (NVFP4):
+ *   codes   uint8 [rows x K/2]: element 2j of a row in bits 0..3 of byte j,
+ *           element 2j+1 in bits 4..7; code = sign<<3 | i, magnitude
+ *           {0,0.5,1,1.5,2,3,4,6}[i] (E2M1).
+ *   scales  uint8 E4M3 (sign 0), one per 16 consecutive elements of a row,
+ *           in the tensor-core scale-factor layout: 512-byte atoms holding
+ *           128 rows x 4 scale columns; atom (r/128, c/4) at byte offset
+ *           ((r/128)*(K/64) + c/4)*512, entry (r, c) inside it at
+ *           (r%32)*16 + ((r%128)/32)*4 + c%4.  Buffer size:
+ *           ceil(rows/128)*128 * K/16 bytes.  Rows are padded to 128.
+ *   s_t     float32 per tensor: s_t = max|x| / 2688 (1 for an all-zero tensor).
+ *   Per 16-block with amax a: sf = E4M3_rne(a * (1/(6 s_t))), d = sf*s_t,
+ *   q = E2M1_rne(x * (1/d)), dequantized value xhat = e2m1(q)*d, residual
+ *   R = x - xhat (binary32 throughout).
+ */
+#ifndef NVFP4_QUADS_H
+#define NVFP4_QUADS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum */
+    NVFP4_ERR_ALIGNMENT = 2,         /* pointer or leading dimension misaligned */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 3, /* shape outside the supported envelope */
+    NVFP4_ERR_CUDA = 4,              /* CUDA runtime / launch failure */
+    NVFP4_ERR_TIMEOUT = 5,           /* a device-side bounded wait ran out */
+    NVFP4_ERR_WORKSPACE = 6          /* workspace missing or too small */
+} nvfp4_status;
+
+/* Library version, e.g. 100 for 0.1.0. */
+NVFP4_API int nvfp4_version(void);
+
+/* Message for the last error returned on the calling thread ("" if none). */
+NVFP4_API const char *nvfp4_last_error_string(void);
+
+/* Synchronously copies a device status word (see dev_status above) to the
+ * host; *status_out receives NVFP4_OK or the device-reported status. */
+NVFP4_API nvfp4_status nvfp4_read_status(const int32_t *dev_status, int32_t *status_out, void *stream);
+
+/* Number of SMs of the current device (used to size persistent grids). */
+NVFP4_API int nvfp4_num_sms(void);
+
+/* --------------------------------------------------------------------------
+ * nvfp4_quantize -- online NVFP4 activation quantization, residual channel
+ * scoring and RAC channel selection (shd-paper.top abstract: activations are
+ * quantized online; gist.science/it 2.2 B: channels with the largest FP4
+ * residual are selected by a top-k binary mask).
+ *
+ * One call runs: (1) per-tensor amax -> s_t (skipped when s_t_in_dev is
+ * given), (2) one streaming pass that writes codes and swizzled scales and
+ * accumulates score[c] = sum_r R[r,c]^2 (binary64 across rows), (3) selection
+ * of the rac_k channels with the largest score (equal scores: lower index
+ * first), returned ascending, (4) the RAC residual operand
+ * r_sel[dst, j] = bf16(R[r, S_j] / s_t) for every output row.
+ *
+ *   x_dev        bf16 [M x K], row stride ldx elements (ldx % 8 == 0).
+ *   M, K         K % 64 == 0, 64 <= K <= 16384; M >= 0.
+ *   m_valid_dev  optional int32 on the device: rows >= *m_valid_dev are
+ *                ignored (absent from amax, scores and outputs).  NULL = M.
+ *   s_t_in_dev   optional float32: use this tensor scale instead of amax.
+ *   s_t_out_dev  float32 [1]: receives s_t (required).
+ *   dst_rows_dev optional int32 [M x fanout]: input row r is written to output
+ *                rows dst_rows[r*fanout + j] (j < fanout); a negative entry
+ *                skips that copy.  NULL: output row = input row, fanout 1.
+ *   M_out        rows of the output arrays (every destination < M_out).
+ *   codes_dev    uint8 [M_out x K/2].
+ *   scales_dev   uint8 swizzled, ceil(M_out/128)*128*K/16 bytes.
+ *   score_dev    optional float64 [K]: receives the channel scores.  Required
+ *                when rac_k > 0.
+ *   rac_k        channels to select, 0 <= rac_k <= min(256, K).
+ *   rac_ld       row stride (elements) of r_sel, rac_ld >= rac_k,
+ *                rac_ld % 64 == 0; columns [rac_k, rac_ld) are written as 0.
+ *   sel_dev      int32 [rac_k]: selected channels, ascending.
+ *   r_sel_dev    bf16 [M_out x rac_ld].
+ *   dev_status   optional int32 status word (see conventions).
+ *   workspace    nvfp4_quantize_workspace_size(M, K) bytes, 16-byte aligned.
+ * Only rows named as destinations are written; other output rows keep their
+ * contents.
+ * -------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K);
+
+NVFP4_API nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
+                            const int32_t *m_valid_dev,
+                            const float *s_t_in_dev, float *s_t_out_dev,
+                            const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
+                            uint8_t *codes_dev, uint8_t *scales_dev,
+                            double *score_dev, int32_t rac_k, int32_t rac_ld,
+                            int32_t *sel_dev, void *r_sel_dev,
+                            int32_t *dev_status, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/* --------------------------------------------------------------------------
+ * nvfp4_qdq_weights -- trainer-side asymmetric QAT weight fake-quantization
+ * (gist.science/it 2.2 A: weights are quantized to NVFP4 and dequantized on
+ * every trainer forward so the trainer sees the rollout's weights; activations
+ * stay BF16), and the rollout engine's weight quantizer.
+ *
+ * G independent tensors w[g] of [rows x cols] bf16 (contiguous, g-major),
+ * each with its own s_t[g] = max|w[g]|/2688.
+ *   w_qdq_dev   optional bf16 [G x rows x cols]: bf16(xhat), nearest even.
+ *   s_t_dev     float32 [G] (required).
+ *   codes_dev   optional uint8 [G x rows x cols/2].
+ *   scales_dev  optional uint8 [G x ceil(rows/128)*128*cols/16], swizzled per
+ *               tensor.
+ * cols % 64 == 0, cols <= 16384, ldx = cols.
+ * -------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_qdq_workspace_size(int64_t G, int64_t rows, int64_t cols);
+
+NVFP4_API nvfp4_status nvfp4_qdq_weights(const void *w_dev, int64_t G, int64_t rows, int64_t cols,
+                               void *w_qdq_dev, float *s_t_dev,
+                               uint8_t *codes_dev, uint8_t *scales_dev,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * moe_route -- top-k_r expert routing of T tokens over E experts and the
+ * expert-grouped routed-row layout used by the grouped GEMMs.
+ *
+ *   logits_dev   float32 [T x E], E <= 256, 1 <= k_r <= min(E, 8).
+ *   topk_idx_dev int32 [T x k_r]: experts by descending logit (equal logits:
+ *                lower expert first).
+ *   topk_gate_dev float32 [T x k_r]: softmax over the k_r selected logits.
+ *   offsets_dev  int32 [E+1]: expert e owns routed rows
+ *                [offsets[e], offsets[e+1]); every segment is padded to a
+ *                multiple of 128 rows; offsets[E] = total padded rows.
+ *   dst_row_dev  int32 [T x k_r]: routed row of (token t, slot j).  Inside
+ *                an expert's segment tokens appear in ascending order.
+ *   row_token_dev int32 [M_pad_max]: token of each routed row, -1 for padding
+ *                and for rows >= offsets[E].
+ *   row_gate_dev float32 [M_pad_max]: gate of each routed row (0 for padding).
+ *   M_pad_max    >= T*k_r + E*127 rounded up to 128.
+ * -------------------------------------------------------------------------- */
+NVFP4_API size_t moe_route_workspace_size(int64_t T, int32_t E);
+
+NVFP4_API nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E, int32_t k_r,
+                       int32_t *topk_idx_dev, float *topk_gate_dev,
+                       int32_t *offsets_dev, int32_t *dst_row_dev,
+                       int32_t *row_token_dev, float *row_gate_dev, int64_t M_pad_max,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * nvfp4_gather_weight_channels -- RAC weight operand: the selected input
+ * channels S of every expert's NVFP4 weight, dequantized without the tensor
+ * scale (e2m1 * sf is exact in bf16):
+ *   w_sel[e, n, j] = bf16(e2m1(q_e[n, S_j]) * sf_e[n, S_j/16])  (j < k)
+ *   w_sel[e, n, j] = 0                                          (k <= j < ld)
+ *   codes_dev  uint8 [E x N x K/2], scales_dev swizzled per expert.
+ *   w_sel_dev  bf16 [E x N x ld], ld % 64 == 0, k <= ld.
+ * -------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_gather_weight_channels(const uint8_t *codes_dev, const uint8_t *scales_dev,
+                                          int32_t E, int64_t N, int64_t K,
+                                          const int32_t *sel_dev, int32_t k, int32_t ld,
+                                          void *w_sel_dev, void *stream);
+
+/* --------------------------------------------------------------------------
+ * moe_w4a4_grouped_gemm_rac -- the native W4A4 block-scaled grouped expert
+ * GEMM with Residual Activation Compensation folded into the same
+ * accumulator (gist.science/it 2.2 B; shd-paper.top abstract: RAC corrects
+ * high-error activation channels while keeping native W4A4 GEMMs).
+ *
+ * For every routed row r of expert e (offsets[e] <= r < offsets[e+1]) and
+ * output feature n:
+ *   D[r,n] = sum_k (e2m1(a)*sfa)[r,k] (e2m1(b_e)*sfb_e)[n,k]      (FP4 MMA)
+ *          + sum_j rho[r,j] w_sel[e,n,j]                          (BF16 MMA)
+ *   y[r,n] = s_a * s_b[e] * D[r,n]
+ * and the epilogue writes y:
+ *   MOE_EPI_STORE_F32    out f32 [M_pad_max x ld_out], rows with
+ *                        row_token < 0 not written.
+ *   MOE_EPI_SWIGLU_BF16  N = 2I (gate rows [0,I), up rows [I,2I) of B);
+ *                        out bf16 [M_pad_max x ld_out]:
+ *                        h[r,i] = bf16(silu(y[r,i]) * y[r,I+i]) for i < I;
+ *                        rows with row_token < 0 (and < offsets[E]) are
+ *                        written as 0.  I % 128 == 0.
+ *   MOE_EPI_SCATTER_ADD_F32  out f32 [T x ld_out]:
+ *                        out[row_token[r], n] += row_gate[r] * y[r,n]
+ *                        (atomic; the caller zeroes out first).
+ *
+ *   a_codes_dev/a_scales_dev  NVFP4 A, rows in routed order, M_pad_max rows.
+ *   a_s_t_dev       float32 [1].
+ *   b_codes_dev/b_scales_dev  NVFP4 B, E tensors of [N x K] (per-expert
+ *                   swizzled scales), b_s_t_dev float32 [E].
+ *   offsets_dev     int32 [E+1] from moe_route (multiples of 128).
+ *   rac_ld          0 (no RAC) or the row stride of rho / w_sel, % 64 == 0,
+ *                   <= 256; rho_dev bf16 [M_pad_max x rac_ld] and
+ *                   w_sel_dev bf16 [E x N x rac_ld].
+ * Shapes: K % 256 == 0, N % 256 == 0 (SWIGLU: I % 128 == 0), M_pad_max % 128
+ * == 0, E <= 256.  Persistent kernel: one CTA per SM.
+ * -------------------------------------------------------------------------- */
+typedef enum {
+    MOE_EPI_STORE_F32 = 0,
+    MOE_EPI_SWIGLU_BF16 = 1,
+    MOE_EPI_SCATTER_ADD_F32 = 2
+} moe_epilogue;
+
+NVFP4_API nvfp4_status moe_w4a4_grouped_gemm_rac(
+    const uint8_t *a_codes_dev, const uint8_t *a_scales_dev, const float *a_s_t_dev,
+    int64_t M_pad_max,
+    const uint8_t *b_codes_dev, const uint8_t *b_scales_dev, const float *b_s_t_dev,
+    int64_t N, int64_t K, int32_t E,
+    const int32_t *offsets_dev,
+    int32_t rac_ld, const void *rho_dev, const void *w_sel_dev,
+    int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev,
+    void *out_dev, int64_t ld_out,
+    int32_t *dev_status, void *stream);
+
+/* --------------------------------------------------------------------------
+ * nvfp4_debug_encode -- runs the library's element and scale encoders on n
+ * arbitrary floats (for validation against an independent definition):
+ *   e2m1_dev[i] = E2M1 code of in[i] (nearest even, saturating, sign bit
+ *                 of in[i]); e4m3_dev[i] = E4M3 code of in[i] >= 0 (nearest
+ *                 even, saturating at 448).  Either output may be NULL.
+ * -------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_debug_encode(const float *in_dev, int64_t n, uint8_t *e2m1_dev, uint8_t *e4m3_dev,
+                                void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_QUADS_H */

@@ -1,0 +1,606 @@
+// quantize.cu -- bandwidth-bound NVFP4 kernels of the QUADS rollout path.
+//
+//   k_amax              per-tensor (per-group) max |x|          (HBM read, 2 B/elem)
+//   k_quantize          one streaming pass: E2M1 codes + swizzled E4M3 scales
+//                       (+ bf16 QDQ values, + per-channel residual score
+//                       partials), fanned out to routed rows   (2 B read,
+//                       0.5625 B/elem written per destination)
+//   k_score_reduce      partial scores -> score[K] (binary64, fixed order)
+//   k_select_topk       radix select of the rac_k largest scores, compacted in
+//                       ascending channel order (one CTA)
+//   k_rac_residual      rho[dst, j] = bf16(R[r, S_j] / s_t)
+//   k_gather_w_channels w_sel[e, n, j] = bf16(e2m1 * sf) of selected channels
+//
+// Layout of k_quantize: a CTA is 8 warps on one 256-channel column chunk and
+// one range of rows.  Each lane owns 8 consecutive channels (one 16-byte
+// load), two lanes form a 16-element block (amax by one xor-shuffle), a warp
+// reads 512 contiguous bytes of a row.  Lanes keep their channels' residual
+// sums across rows (binary32 for 4 rows, then binary64), the CTA reduces its
+// 8 warps in shared memory and writes one partial per channel; partials are
+// summed in a fixed order by k_score_reduce, so scores are deterministic.
+#include "common.cuh"
+
+#include <algorithm>
+
+namespace nvfp4 {
+
+constexpr int QTHREADS = 256;
+constexpr int QCHUNK = 256;           // channels per CTA column chunk
+constexpr int SCORE_FLUSH = 4;        // rows summed in binary32 before binary64
+
+// -------------------------------------------------------------------- amax
+
+__global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16 *__restrict__ x, int64_t ldx,
+                                              int64_t M, int64_t K, const int32_t *__restrict__ m_valid,
+                                              int64_t group_stride, unsigned int *__restrict__ amax_bits)
+{
+    int64_t Me = M;
+    if (m_valid) Me = min(Me, (int64_t)max(*m_valid, 0));
+    const __nv_bfloat16 *xg = x + (int64_t)blockIdx.y * group_stride;
+    const int vec_per_row = (int)(K / 8);
+    float m = 0.0f;
+    // each warp sweeps whole rows; rows are strided over all warps of the grid
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t r = gw; r < Me; r += nw) {
+        const uint4 *row = reinterpret_cast<const uint4 *>(xg + r * ldx);
+        for (int v = lane; v < vec_per_row; v += 32) {
+            uint4 u = __ldg(row + v);
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(u.x)), fabsf(bf16hi(u.x))),
+                               fmaxf(fabsf(bf16lo(u.y)), fabsf(bf16hi(u.y)))));
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(u.z)), fabsf(bf16hi(u.z))),
+                               fmaxf(fabsf(bf16lo(u.w)), fabsf(bf16hi(u.w)))));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __shared__ float wm[8];
+    if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = wm[0];
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) b = fmaxf(b, wm[w]);
+        // non-negative floats order like their bit patterns
+        atomicMax(amax_bits + blockIdx.y, __float_as_uint(b));
+    }
+}
+
+// --------------------------------------------------------------- quantize
+
+struct QuantParams {
+    const __nv_bfloat16 *x;
+    int64_t ldx, M, K;
+    const int32_t *m_valid;
+    const float *s_t_in;             // per group, or null
+    const unsigned int *amax_bits;   // per group, used when s_t_in is null
+    float *s_t_out;                  // per group
+    const int32_t *dst_rows;
+    int fanout;
+    uint8_t *codes;
+    uint8_t *scales;
+    __nv_bfloat16 *qdq;
+    double *partials;                // [gridDim.y x K]
+    int64_t rows_per_cta;
+    int64_t x_gstride, codes_gstride, scales_gstride, qdq_gstride;
+};
+
+template <bool SCORE>
+__global__ void __launch_bounds__(QTHREADS) k_quantize(QuantParams p)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = blockIdx.z;
+    const int64_t K = p.K;
+    const int64_t c = (int64_t)blockIdx.x * QCHUNK + lane * 8;   // first channel of this lane
+    const bool active = c < K;
+
+    float s_t = p.s_t_in ? p.s_t_in[g] : tensor_scale_from_amax(__uint_as_float(p.amax_bits[g]));
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.s_t_out) p.s_t_out[g] = s_t;
+    const float r6 = block_r6(s_t);
+
+    int64_t Me = p.M;
+    if (p.m_valid) Me = min(Me, (int64_t)max(*p.m_valid, 0));
+    const int64_t r0 = (int64_t)blockIdx.y * p.rows_per_cta;
+    const int64_t r1 = min(Me, r0 + p.rows_per_cta);
+
+    const __nv_bfloat16 *xg = p.x + g * p.x_gstride;
+    uint8_t *codes = p.codes ? p.codes + g * p.codes_gstride : nullptr;
+    uint8_t *scales = p.scales ? p.scales + g * p.scales_gstride : nullptr;
+    __nv_bfloat16 *qdq = p.qdq ? p.qdq + g * p.qdq_gstride : nullptr;
+
+    float acc32[8];
+    double acc64[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { acc32[i] = 0.0f; acc64[i] = 0.0; }
+    int since_flush = 0;
+
+    const int64_t kb0 = c >> 4;                 // first block of the 4-block group (lanes 8j)
+    for (int64_t r = r0 + warp; r < r1; r += QTHREADS / 32) {
+        float v[8];
+        if (active) {
+            uint4 u = __ldg(reinterpret_cast<const uint4 *>(xg + r * p.ldx + c));
+            v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+            v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+        }
+        float m = fabsf(v[0]);
+#pragma unroll
+        for (int i = 1; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        BlockScale bs = block_scale(m, s_t, r6);
+        float xh[8];
+        uint32_t cw = quant8(v, bs, xh);
+
+        // gather the 4 scale codes of blocks kb0..kb0+3 onto lanes 8j
+        uint32_t s1 = __shfl_down_sync(0xffffffffu, bs.sf_code, 2);
+        uint32_t s2 = __shfl_down_sync(0xffffffffu, bs.sf_code, 4);
+        uint32_t s3 = __shfl_down_sync(0xffffffffu, bs.sf_code, 6);
+        uint32_t sw = bs.sf_code | (s1 << 8) | (s2 << 16) | (s3 << 24);
+
+        if (active) {
+            if (SCORE) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float R = __fsub_rn(v[i], xh[i]);
+                    acc32[i] = fmaf(R, R, acc32[i]);
+                }
+                if (++since_flush == SCORE_FLUSH) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) { acc64[i] += (double)acc32[i]; acc32[i] = 0.0f; }
+                    since_flush = 0;
+                }
+            }
+            if (qdq) {
+                uint4 o;
+                o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[0])) |
+                      ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[1])) << 16);
+                o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[2])) |
+                      ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[3])) << 16);
+                o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[4])) |
+                      ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[5])) << 16);
+                o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[6])) |
+                      ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[7])) << 16);
+                *reinterpret_cast<uint4 *>(qdq + r * K + c) = o;
+            }
+            if (codes) {
+                const int nd = p.dst_rows ? p.fanout : 1;
+                for (int j = 0; j < nd; ++j) {
+                    int64_t dst = p.dst_rows ? (int64_t)p.dst_rows[r * p.fanout + j] : r;
+                    if (dst < 0) continue;
+                    *reinterpret_cast<uint32_t *>(codes + dst * (K >> 1) + (c >> 1)) = cw;
+                    if ((lane & 7) == 0)
+                        *reinterpret_cast<uint32_t *>(scales + sf_offset(dst, kb0, K)) = sw;
+                }
+            }
+        }
+    }
+
+    if (SCORE) {
+        __shared__ double red[QTHREADS / 32][QCHUNK];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[warp][lane * 8 + i] = acc64[i] + (double)acc32[i];
+        __syncthreads();
+        int64_t ch = (int64_t)blockIdx.x * QCHUNK + threadIdx.x;
+        if (ch < K) {
+            double s = 0.0;
+#pragma unroll
+            for (int w = 0; w < QTHREADS / 32; ++w) s += red[w][threadIdx.x];
+            p.partials[(int64_t)blockIdx.y * K + ch] = s;
+        }
+    }
+}
+
+// ----------------------------------------------------------- score reduce
+
+__global__ void k_score_reduce(const double *__restrict__ partials, int64_t P, int64_t K,
+                               double *__restrict__ score)
+{
+    int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= K) return;
+    double s = 0.0;
+    for (int64_t q = 0; q < P; ++q) s += partials[q * K + c];
+    score[c] = s;
+}
+
+// ---------------------------------------------------------------- top-k
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int *smem_warp, int &total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    __syncthreads();
+    if (lane == 31) smem_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? smem_warp[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int t = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += t;
+        }
+        if (lane < nw) smem_warp[lane] = wi - w;     // exclusive warp offsets
+        if (lane == nw - 1) smem_warp[32] = wi;      // total
+    }
+    __syncthreads();
+    int r = smem_warp[warp] + incl - v;
+    total = smem_warp[32];
+    return r;
+}
+
+// One CTA of 1024 threads.  Scores are non-negative binary64, whose bit
+// patterns order like their values; an 8-pass MSB-first radix select finds
+// the k-th largest key, then channels are taken in ascending index order:
+// every key above it, and the lowest-index keys equal to it.
+__global__ void __launch_bounds__(1024) k_select_topk(const double *__restrict__ score, int K, int k,
+                                                      int32_t *__restrict__ sel)
+{
+    extern __shared__ unsigned long long keys[];
+    __shared__ unsigned int hist[256];
+    __shared__ int scan_tmp[33];
+    __shared__ int s_digit, s_rem;
+    const int tid = threadIdx.x;
+    if (k <= 0) return;
+    for (int i = tid; i < K; i += blockDim.x) keys[i] = (unsigned long long)__double_as_longlong(score[i]);
+    if (tid == 0) s_rem = k;
+    __syncthreads();
+
+    unsigned long long prefix = 0ull, mask = 0ull;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < K; i += blockDim.x) {
+            unsigned long long key = keys[i];
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255ull], 1u);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int rem = s_rem;
+            unsigned int above = 0;
+            int d = 255;
+            for (; d > 0; --d) {
+                if (above + hist[d] >= (unsigned)rem) break;
+                above += hist[d];
+            }
+            s_digit = d;
+            s_rem = rem - (int)above;
+        }
+        __syncthreads();
+        prefix |= (unsigned long long)s_digit << shift;
+        mask |= 0xFFull << shift;
+    }
+    const unsigned long long kth = prefix;
+    const int take_eq = s_rem;          // keys equal to kth to take, lowest index first
+
+    // contiguous ranges per thread
+    const int per = (K + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(K, tid * per), i1 = min(K, i0 + per);
+    int n_eq = 0;
+    for (int i = i0; i < i1; ++i) n_eq += (keys[i] == kth);
+    int tot;
+    int eq_before = block_exclusive_scan(n_eq, scan_tmp, tot);
+    int n_take = 0;
+    {
+        int e = eq_before;
+        for (int i = i0; i < i1; ++i) {
+            unsigned long long key = keys[i];
+            if (key > kth) ++n_take;
+            else if (key == kth) { if (e < take_eq) ++n_take; ++e; }
+        }
+    }
+    int take_before = block_exclusive_scan(n_take, scan_tmp, tot);
+    {
+        int e = eq_before, pos = take_before;
+        for (int i = i0; i < i1; ++i) {
+            unsigned long long key = keys[i];
+            bool t = false;
+            if (key > kth) t = true;
+            else if (key == kth) { t = e < take_eq; ++e; }
+            if (t && pos < k) sel[pos++] = i;
+        }
+    }
+}
+
+// --------------------------------------------------------- RAC residual
+
+// One warp per input row; lane j handles selected channel S_j.  The block of
+// S_j is re-quantized from x with the same arithmetic as k_quantize (one lane
+// takes the whole 16-block max), giving the residual bit for bit.
+__global__ void __launch_bounds__(256) k_rac_residual(
+    const __nv_bfloat16 *__restrict__ x, int64_t ldx, int64_t M, int64_t K,
+    const int32_t *__restrict__ m_valid, const float *__restrict__ s_t_ptr,
+    const int32_t *__restrict__ sel, int k, int ld,
+    const int32_t *__restrict__ dst_rows, int fanout, __nv_bfloat16 *__restrict__ r_sel)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    int64_t Me = M;
+    if (m_valid) Me = min(Me, (int64_t)max(*m_valid, 0));
+    if (r >= Me) return;
+    const float s_t = *s_t_ptr;
+    const float r6 = block_r6(s_t);
+    const int nd = dst_rows ? fanout : 1;
+    for (int j = lane; j < ld; j += 32) {
+        __nv_bfloat16 outv = __float2bfloat16_rn(0.0f);
+        if (j < k) {
+            const int64_t ch = sel[j];
+            const __nv_bfloat16 *blk = x + r * ldx + (ch & ~15ll);
+            uint4 u0 = __ldg(reinterpret_cast<const uint4 *>(blk));
+            uint4 u1 = __ldg(reinterpret_cast<const uint4 *>(blk + 8));
+            uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            float m = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[i])), fabsf(bf16hi(w[i]))));
+            BlockScale bs = block_scale(m, s_t, r6);
+            int idx = (int)(ch & 15);
+            uint32_t word = w[idx >> 1];
+            float xv = (idx & 1) ? bf16hi(word) : bf16lo(word);
+            float R = __fsub_rn(xv, quant1_xhat(xv, bs));
+            outv = __float2bfloat16_rn(__fdiv_rn(R, s_t));
+        }
+        for (int d = 0; d < nd; ++d) {
+            int64_t dst = dst_rows ? (int64_t)dst_rows[r * fanout + d] : r;
+            if (dst >= 0) r_sel[dst * ld + j] = outv;
+        }
+    }
+}
+
+// --------------------------------------------------- weight channel gather
+
+__global__ void k_gather_w_channels(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                                    int64_t E, int64_t N, int64_t K, const int32_t *__restrict__ sel,
+                                    int k, int ld, __nv_bfloat16 *__restrict__ out)
+{
+    const int64_t total = E * N * ld;
+    const int64_t sf_per_e = sf_bytes(N, K);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int64_t j = i % ld;
+        int64_t en = i / ld;
+        int64_t n = en % N, e = en / N;
+        float v = 0.0f;
+        if (j < k) {
+            int64_t ch = sel[j];
+            uint32_t byte = codes[en * (K >> 1) + (ch >> 1)];
+            uint32_t nib = (ch & 1) ? (byte >> 4) : (byte & 15u);
+            float q = e2m1x2_to_f32(nib).x;
+            float sf = e4m3_to_f32(scales[e * sf_per_e + sf_offset(n, ch >> 4, K)]);
+            v = __fmul_rn(q, sf);   // exact: <= 6 significant bits
+        }
+        out[i] = __float2bfloat16_rn(v);
+    }
+}
+
+// --------------------------------------------------------------- helpers
+
+static int64_t pick_rows_per_cta(int64_t M, int64_t nchunks, int64_t groups)
+{
+    // aim for ~4 CTAs per SM over the whole grid, at least 8 rows per CTA
+    int64_t target = (int64_t)num_sms() * 4;
+    int64_t per_group = std::max<int64_t>(1, target / std::max<int64_t>(1, nchunks * groups));
+    int64_t rpc = (M + per_group - 1) / per_group;
+    rpc = std::max<int64_t>(rpc, 8);
+    return rpc;
+}
+
+static int64_t row_groups(int64_t M, int64_t rpc) { return std::max<int64_t>(1, (M + rpc - 1) / rpc); }
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+// Workspace: [0,256) amax slots (64 groups of 4 B... one slot used), then the
+// score partials [P x K] binary64, then score[K] when the caller gave none.
+extern "C" size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K)
+{
+    if (M < 0 || K <= 0) return 0;
+    int64_t nch = (K + QCHUNK - 1) / QCHUNK;
+    int64_t rpc = pick_rows_per_cta(M, nch, 1);
+    int64_t P = row_groups(M, rpc);
+    return 256 + (size_t)(P * K + K) * sizeof(double);
+}
+
+extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
+                                       const int32_t *m_valid_dev,
+                                       const float *s_t_in_dev, float *s_t_out_dev,
+                                       const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
+                                       uint8_t *codes_dev, uint8_t *scales_dev,
+                                       double *score_dev, int32_t rac_k, int32_t rac_ld,
+                                       int32_t *sel_dev, void *r_sel_dev,
+                                       int32_t *dev_status, void *workspace, size_t workspace_bytes,
+                                       void *stream)
+{
+    (void)dev_status;
+    cudaStream_t st = (cudaStream_t)stream;
+    NVFP4_REQUIRE(M >= 0 && K > 0 && M_out >= 0, NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: bad sizes");
+    NVFP4_REQUIRE(s_t_out_dev && (M == 0 || x_dev) && (M_out == 0 || (codes_dev && scales_dev)),
+                  NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: x, s_t_out, codes and scales are required");
+    NVFP4_REQUIRE(K % 64 == 0 && K <= 16384, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_quantize: K must be a multiple of 64 and <= 16384 (K=%lld)", (long long)K);
+    NVFP4_REQUIRE(ldx >= K && ldx % 8 == 0, NVFP4_ERR_ALIGNMENT, "nvfp4_quantize: ldx must be >= K and a multiple of 8");
+    NVFP4_REQUIRE(aligned16(x_dev) && aligned16(codes_dev) && aligned16(scales_dev),
+                  NVFP4_ERR_ALIGNMENT,
+                  "nvfp4_quantize: x, codes and scales must be 16-byte aligned");
+    NVFP4_REQUIRE(dst_rows_dev == nullptr || fanout >= 1, NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_quantize: fanout must be >= 1 with dst_rows");
+    NVFP4_REQUIRE(dst_rows_dev != nullptr || M_out >= M, NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_quantize: M_out must be >= M without dst_rows");
+    NVFP4_REQUIRE(rac_k >= 0 && rac_k <= 256 && rac_k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_quantize: rac_k must be in [0, min(256, K)]");
+    if (rac_k > 0) {
+        NVFP4_REQUIRE(sel_dev && r_sel_dev, NVFP4_ERR_INVALID_ARG,
+                      "nvfp4_quantize: rac_k > 0 needs sel and r_sel");
+        NVFP4_REQUIRE(rac_ld >= rac_k && rac_ld % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                      "nvfp4_quantize: rac_ld must be >= rac_k and a multiple of 64");
+        NVFP4_REQUIRE(aligned16(r_sel_dev), NVFP4_ERR_ALIGNMENT, "nvfp4_quantize: r_sel must be 16-byte aligned");
+    }
+    const bool want_score = score_dev != nullptr || rac_k > 0;
+    size_t need = nvfp4_quantize_workspace_size(M, K);
+    NVFP4_REQUIRE(workspace && workspace_bytes >= need && aligned16(workspace), NVFP4_ERR_WORKSPACE,
+                  "nvfp4_quantize: workspace of %zu bytes (16-byte aligned) required", need);
+
+    unsigned int *amax_bits = reinterpret_cast<unsigned int *>(workspace);
+    const int64_t nch = (K + QCHUNK - 1) / QCHUNK;
+    const int64_t rpc = pick_rows_per_cta(M, nch, 1);
+    const int64_t P = row_groups(M, rpc);
+    double *partials = reinterpret_cast<double *>(reinterpret_cast<char *>(workspace) + 256);
+    double *score = score_dev ? score_dev : partials + P * K;
+
+    if (!s_t_in_dev) {
+        if (cudaMemsetAsync(amax_bits, 0, 4, st) != cudaSuccess) return check_launch("nvfp4_quantize: memset");
+        if (M > 0) {
+            int blocks = (int)std::min<int64_t>((int64_t)num_sms() * 8, std::max<int64_t>(1, (M * K / 8 + 255) / 256));
+            k_amax<<<dim3(blocks, 1), 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, 0, amax_bits);
+            if (check_launch("k_amax") != NVFP4_OK) return NVFP4_ERR_CUDA;
+        }
+    }
+    QuantParams p{};
+    p.x = (const __nv_bfloat16 *)x_dev;
+    p.ldx = ldx; p.M = M; p.K = K;
+    p.m_valid = m_valid_dev;
+    p.s_t_in = s_t_in_dev;
+    p.amax_bits = amax_bits;
+    p.s_t_out = s_t_out_dev;
+    p.dst_rows = dst_rows_dev;
+    p.fanout = dst_rows_dev ? fanout : 1;
+    p.codes = codes_dev;
+    p.scales = scales_dev;
+    p.qdq = nullptr;
+    p.partials = partials;
+    p.rows_per_cta = rpc;
+    dim3 grid((unsigned)nch, (unsigned)P, 1);
+    if (want_score) k_quantize<true><<<grid, QTHREADS, 0, st>>>(p);
+    else k_quantize<false><<<grid, QTHREADS, 0, st>>>(p);
+    if (check_launch("k_quantize") != NVFP4_OK) return NVFP4_ERR_CUDA;
+
+    if (want_score) {
+        k_score_reduce<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(partials, P, K, score);
+        if (check_launch("k_score_reduce") != NVFP4_OK) return NVFP4_ERR_CUDA;
+    }
+    if (rac_k > 0) {
+        size_t smem = (size_t)K * sizeof(unsigned long long);
+        static bool attr_set = false;
+        if (!attr_set) {
+            cudaFuncSetAttribute(k_select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, 16384 * 8);
+            attr_set = true;
+        }
+        k_select_topk<<<1, 1024, smem, st>>>(score, (int)K, rac_k, sel_dev);
+        if (check_launch("k_select_topk") != NVFP4_OK) return NVFP4_ERR_CUDA;
+        if (M > 0) {
+            const float *s_t_used = s_t_in_dev ? s_t_in_dev : s_t_out_dev;
+            unsigned blocks = (unsigned)((M + 7) / 8);
+            k_rac_residual<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, s_t_used,
+                                                   sel_dev, rac_k, rac_ld, dst_rows_dev,
+                                                   dst_rows_dev ? fanout : 1, (__nv_bfloat16 *)r_sel_dev);
+            if (check_launch("k_rac_residual") != NVFP4_OK) return NVFP4_ERR_CUDA;
+        }
+    }
+    return NVFP4_OK;
+}
+
+extern "C" size_t nvfp4_qdq_workspace_size(int64_t G, int64_t rows, int64_t cols)
+{
+    (void)rows; (void)cols;
+    if (G <= 0) return 0;
+    return (size_t)(((G * 4) + 255) / 256 * 256);
+}
+
+extern "C" nvfp4_status nvfp4_qdq_weights(const void *w_dev, int64_t G, int64_t rows, int64_t cols,
+                                          void *w_qdq_dev, float *s_t_dev,
+                                          uint8_t *codes_dev, uint8_t *scales_dev,
+                                          void *workspace, size_t workspace_bytes, void *stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    NVFP4_REQUIRE(w_dev && s_t_dev, NVFP4_ERR_INVALID_ARG, "nvfp4_qdq_weights: w and s_t are required");
+    NVFP4_REQUIRE(G >= 1 && G <= 65535 && rows >= 1 && cols >= 1, NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_qdq_weights: bad sizes");
+    NVFP4_REQUIRE(cols % 64 == 0 && cols <= 16384, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_qdq_weights: cols must be a multiple of 64 and <= 16384");
+    NVFP4_REQUIRE((codes_dev == nullptr) == (scales_dev == nullptr), NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_qdq_weights: codes and scales go together");
+    NVFP4_REQUIRE(aligned16(w_dev) && (!w_qdq_dev || aligned16(w_qdq_dev)) &&
+                  (!codes_dev || (aligned16(codes_dev) && aligned16(scales_dev))), NVFP4_ERR_ALIGNMENT,
+                  "nvfp4_qdq_weights: pointers must be 16-byte aligned");
+    size_t need = nvfp4_qdq_workspace_size(G, rows, cols);
+    NVFP4_REQUIRE(workspace && workspace_bytes >= need && aligned16(workspace), NVFP4_ERR_WORKSPACE,
+                  "nvfp4_qdq_weights: workspace of %zu bytes required", need);
+    unsigned int *amax_bits = reinterpret_cast<unsigned int *>(workspace);
+    if (cudaMemsetAsync(amax_bits, 0, (size_t)G * 4, st) != cudaSuccess) return check_launch("qdq memset");
+    const int64_t per_group = rows * cols;
+    {
+        int64_t want = std::max<int64_t>(1, (int64_t)num_sms() * 8 / G);
+        int blocks = (int)std::min<int64_t>(want, std::max<int64_t>(1, (per_group / 8 + 255) / 256));
+        k_amax<<<dim3(blocks, (unsigned)G), 256, 0, st>>>((const __nv_bfloat16 *)w_dev, cols, rows, cols,
+                                                          nullptr, per_group, amax_bits);
+        if (check_launch("k_amax (qdq)") != NVFP4_OK) return NVFP4_ERR_CUDA;
+    }
+    const int64_t nch = (cols + QCHUNK - 1) / QCHUNK;
+    const int64_t rpc = pick_rows_per_cta(rows, nch, G);
+    QuantParams p{};
+    p.x = (const __nv_bfloat16 *)w_dev;
+    p.ldx = cols; p.M = rows; p.K = cols;
+    p.amax_bits = amax_bits;
+    p.s_t_out = s_t_dev;
+    p.fanout = 1;
+    p.codes = codes_dev;
+    p.scales = scales_dev;
+    p.qdq = (__nv_bfloat16 *)w_qdq_dev;
+    p.rows_per_cta = rpc;
+    p.x_gstride = per_group;
+    p.codes_gstride = per_group / 2;
+    p.scales_gstride = sf_bytes(rows, cols);
+    p.qdq_gstride = per_group;
+    dim3 grid((unsigned)nch, (unsigned)row_groups(rows, rpc), (unsigned)G);
+    k_quantize<false><<<grid, QTHREADS, 0, st>>>(p);
+    return check_launch("k_quantize (qdq)");
+}
+
+extern "C" nvfp4_status nvfp4_gather_weight_channels(const uint8_t *codes_dev, const uint8_t *scales_dev,
+                                                     int32_t E, int64_t N, int64_t K,
+                                                     const int32_t *sel_dev, int32_t k, int32_t ld,
+                                                     void *w_sel_dev, void *stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    NVFP4_REQUIRE(codes_dev && scales_dev && w_sel_dev && (k == 0 || sel_dev), NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_gather_weight_channels: null pointer");
+    NVFP4_REQUIRE(E >= 1 && N >= 1 && K >= 64 && K % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_gather_weight_channels: bad shape");
+    NVFP4_REQUIRE(k >= 0 && k <= ld && ld % 64 == 0 && ld <= 256 && k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_gather_weight_channels: need 0 <= k <= ld <= 256, ld % 64 == 0");
+    int64_t total = (int64_t)E * N * ld;
+    int blocks = (int)std::min<int64_t>((int64_t)num_sms() * 16, (total + 255) / 256);
+    k_gather_w_channels<<<blocks, 256, 0, st>>>(codes_dev, scales_dev, E, N, K, sel_dev, k, ld,
+                                                (__nv_bfloat16 *)w_sel_dev);
+    return check_launch("k_gather_w_channels");
+}
+
+// ------------------------------------------------------- conversion probe
+
+namespace nvfp4 {
+__global__ void k_debug_encode(const float *__restrict__ in, int64_t n, uint8_t *__restrict__ e2m1,
+                               uint8_t *__restrict__ e4m3)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        float v = in[i];
+        if (e2m1) e2m1[i] = (uint8_t)cvt_e2m1x2(v, 0.0f);
+        if (e4m3) e4m3[i] = (uint8_t)cvt_e4m3(v);
+    }
+}
+}  // namespace nvfp4
+
+extern "C" nvfp4_status nvfp4_debug_encode(const float *in_dev, int64_t n, uint8_t *e2m1_dev, uint8_t *e4m3_dev,
+                                           void *stream)
+{
+    NVFP4_REQUIRE(in_dev && n >= 0, NVFP4_ERR_INVALID_ARG, "nvfp4_debug_encode: bad arguments");
+    if (n == 0) return NVFP4_OK;
+    int blocks = (int)std::min<int64_t>((int64_t)num_sms() * 8, (n + 255) / 256);
+    k_debug_encode<<<blocks, 256, 0, (cudaStream_t)stream>>>(in_dev, n, e2m1_dev, e4m3_dev);
+    return check_launch("k_debug_encode");
+}

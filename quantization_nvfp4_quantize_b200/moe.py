@@ -1,0 +1,127 @@
+"""The QUADS rollout MoE expert layer on the library's kernels.
+
+One forward = the whole hot path (QUADS pages: gist.science/it sections 1
+and 2.2 B; shd-paper.top abstract):
+
+  1. moe_route                 top-k_r routing, expert-grouped padded row layout
+  2. nvfp4_quantize(X)         amax -> s_x, codes/scales written to every routed
+                               row of each token, channel scores, top-k S_x,
+                               RAC residual rho_x for every routed row
+  3. gather_weight_channels    W13q[:, :, S_x] as bf16 (e2m1 * sf)
+  4. grouped GEMM (gate/up)    W4A4 + RAC, epilogue SwiGLU -> h bf16
+  5. nvfp4_quantize(h)         over the valid routed rows: s_h, codes, S_h, rho_h
+  6. gather_weight_channels    W2q[:, :, S_h]
+  7. grouped GEMM (down)       W4A4 + RAC, epilogue router-weighted scatter-add
+                               into Y [T x H] fp32
+
+Weights are quantized to NVFP4 once at construction (the rollout engine holds
+NVFP4 weights).  All buffers are allocated once; ``forward`` launches only the
+library's kernels plus one memset of Y.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import api
+
+
+class MoELayerW4A4:
+    def __init__(self, w13: torch.Tensor, w2: torch.Tensor, tokens: int, topk: int, rac_k: int):
+        assert w13.dtype == torch.bfloat16 and w2.dtype == torch.bfloat16
+        E, N13, H = w13.shape
+        E2, H2, I = w2.shape
+        assert E2 == E and H2 == H and N13 == 2 * I
+        dev = w13.device
+        self.E, self.H, self.I, self.T, self.k_r = E, H, I, tokens, topk
+        self.rac_k = rac_k
+        self.rac_ld = -(-rac_k // 64) * 64 if rac_k else 0
+        _, self.s13, self.c13, self.sf13 = api.qdq_weights(w13, want_qdq=False, want_packed=True)
+        _, self.s2, self.c2, self.sf2 = api.qdq_weights(w2, want_qdq=False, want_packed=True)
+        self.m_pad = api.padded_rows_bound(tokens, topk, E)
+        mp, ld = self.m_pad, max(self.rac_ld, 1)
+        self.xq = api.Quantized(
+            codes=torch.empty(mp, H // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(api.scale_bytes(mp, H), dtype=torch.uint8, device=dev),
+            s_t=torch.empty(1, dtype=torch.float32, device=dev),
+            score=torch.empty(H, dtype=torch.float64, device=dev),
+            sel=torch.empty(max(rac_k, 1), dtype=torch.int32, device=dev),
+            r_sel=torch.empty(mp, ld, dtype=torch.bfloat16, device=dev))
+        self.hq = api.Quantized(
+            codes=torch.empty(mp, I // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(api.scale_bytes(mp, I), dtype=torch.uint8, device=dev),
+            s_t=torch.empty(1, dtype=torch.float32, device=dev),
+            score=torch.empty(I, dtype=torch.float64, device=dev),
+            sel=torch.empty(max(rac_k, 1), dtype=torch.int32, device=dev),
+            r_sel=torch.empty(mp, ld, dtype=torch.bfloat16, device=dev))
+        self.w_sel13 = torch.empty(E, 2 * I, ld, dtype=torch.bfloat16, device=dev)
+        self.w_sel2 = torch.empty(E, H, ld, dtype=torch.bfloat16, device=dev)
+        self.h = torch.empty(mp, I, dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty(tokens, H, dtype=torch.float32, device=dev)
+        lib = api._lib.load()
+        self.ws_x = api._ws(lib.nvfp4_quantize_workspace_size(tokens, H), dev)
+        self.ws_h = api._ws(lib.nvfp4_quantize_workspace_size(mp, I), dev)
+        self.routing = None
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor) -> torch.Tensor:
+        E, H, I, k = self.E, self.H, self.I, self.rac_k
+        r = api.route(logits, self.k_r, self.m_pad) if self.routing is None else self._route_into(logits)
+        self.routing = r
+        api.quantize(x, rac_k=k, rac_ld=self.rac_ld, dst_rows=r.dst_row, fanout=self.k_r, m_out=self.m_pad,
+                     out=self.xq, workspace=self.ws_x)
+        if k:
+            api.gather_weight_channels(self.c13, self.sf13, 2 * I, H, self.xq.sel, k, self.rac_ld, out=self.w_sel13)
+        api.grouped_gemm(self.xq.codes, self.xq.scales, self.xq.s_t, self.m_pad, self.c13, self.sf13, self.s13,
+                         2 * I, H, E, r.offsets, rac_ld=self.rac_ld if k else 0, rho=self.xq.r_sel,
+                         w_sel=self.w_sel13, epilogue=api.EPI_SWIGLU_BF16, row_token=r.row_token,
+                         row_gate=r.row_gate, out=self.h)
+        api.quantize(self.h, rac_k=k, rac_ld=self.rac_ld, m_out=self.m_pad, m_valid=r.offsets[E:],
+                     out=self.hq, workspace=self.ws_h)
+        if k:
+            api.gather_weight_channels(self.c2, self.sf2, H, I, self.hq.sel, k, self.rac_ld, out=self.w_sel2)
+        self.y.zero_()
+        api.grouped_gemm(self.hq.codes, self.hq.scales, self.hq.s_t, self.m_pad, self.c2, self.sf2, self.s2,
+                         H, I, E, r.offsets, rac_ld=self.rac_ld if k else 0, rho=self.hq.r_sel, w_sel=self.w_sel2,
+                         epilogue=api.EPI_SCATTER_ADD_F32, row_token=r.row_token, row_gate=r.row_gate, out=self.y)
+        return self.y
+
+    def _route_into(self, logits):
+        lib = api._lib.load()
+        r = self.routing
+        T, E = logits.shape
+        ws = getattr(self, "_ws_route", None)
+        if ws is None:
+            ws = self._ws_route = api._ws(lib.moe_route_workspace_size(T, E), logits.device)
+        api.check(lib.moe_route(api._p(logits), T, E, self.k_r, api._p(r.topk_idx), api._p(r.topk_gate),
+                                api._p(r.offsets), api._p(r.dst_row), api._p(r.row_token), api._p(r.row_gate),
+                                r.m_pad_max, api._p(ws), ws.numel(), api._stream(logits.device)))
+        return r
+
+
+class DenseLayerW4A4:
+    """Single dense W4A4 + RAC layer: Y = Xq Wq^T + RAC, fp32 out (one expert,
+    identity routing)."""
+
+    def __init__(self, w: torch.Tensor, tokens: int, rac_k: int):
+        N, K = w.shape
+        self.N, self.K, self.T, self.rac_k = N, K, tokens, rac_k
+        self.rac_ld = -(-rac_k // 64) * 64 if rac_k else 0
+        _, self.s_w, self.c_w, self.sf_w = api.qdq_weights(w.unsqueeze(0).contiguous(), want_qdq=False,
+                                                           want_packed=True)
+        self.m_pad = api.padded_rows_bound(tokens, 1, 1)
+        dev = w.device
+        self.out = torch.empty(self.m_pad, N, dtype=torch.float32, device=dev)
+        self.w_sel = torch.empty(1, N, max(self.rac_ld, 1), dtype=torch.bfloat16, device=dev)
+        self.logits = torch.zeros(tokens, 1, dtype=torch.float32, device=dev)
+
+    def forward(self, x: torch.Tensor):
+        r = api.route(self.logits, 1, self.m_pad)
+        self.routing = r
+        xq = api.quantize(x, rac_k=self.rac_k, rac_ld=self.rac_ld, dst_rows=r.dst_row, fanout=1, m_out=self.m_pad)
+        self.xq = xq
+        if self.rac_k:
+            api.gather_weight_channels(self.c_w, self.sf_w, self.N, self.K, xq.sel, self.rac_k, self.rac_ld,
+                                       out=self.w_sel)
+        api.grouped_gemm(xq.codes, xq.scales, xq.s_t, self.m_pad, self.c_w, self.sf_w, self.s_w, self.N, self.K, 1,
+                         r.offsets, rac_ld=self.rac_ld, rho=xq.r_sel, w_sel=self.w_sel,
+                         epilogue=api.EPI_STORE_F32, row_token=r.row_token, row_gate=r.row_gate, out=self.out)
+        return self.out[: self.T]

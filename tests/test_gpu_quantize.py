@@ -1,0 +1,208 @@
+"""GPU parity of the bandwidth kernels (through the C ABI) against the oracle:
+encoders, quantize + scores + selection + RAC residual, weight QDQ, routing,
+weight channel gather.  Codes, scale bytes, tensor scales, selected channel
+sets (outside the 1e-6 tie window), RAC residuals and QDQ values are
+bit-exact; scores agree to 5.5e-7 relative (binary32 partial sums of at most
+4 rows, binary64 above)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import np_u16, to_bf16_dev, check_selection, unswizzle
+from quantization_nvfp4_quantize_b200 import api
+
+pytestmark = pytest.mark.gpu
+
+SCORE_RTOL = 5.5e-7
+
+
+def gen_x(rng, M, K, outliers=4, scale=1.0):
+    x = rng.standard_normal((M, K)).astype(np.float32) * scale
+    if outliers and K:
+        ch = rng.choice(K, size=min(outliers, K), replace=False)
+        x[:, ch] *= np.exp(2.0 + 0.5 * rng.standard_normal(len(ch))).astype(np.float32)
+    return oracle.f32_to_bf16(x)
+
+
+def test_hw_encoders_match_oracle(cuda):
+    h = np.arange(65536, dtype=np.uint32)
+    f = (h << 16).view(np.float32)
+    f = f[np.isfinite(f)]
+    rng = np.random.default_rng(0)
+    grid = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    mids = np.concatenate([grid, np.nextafter(grid, np.float32(0)), np.nextafter(grid, np.float32(9))])
+    r = rng.uniform(-8, 8, 1_000_000).astype(np.float32)
+    vals = np.concatenate([f, mids, -mids, r]).astype(np.float32)
+    e2, _ = api.debug_encode(torch.from_numpy(vals).to(cuda))
+    ref2 = oracle.e2m1_encode(vals)
+    bad = np.nonzero(e2.cpu().numpy() != ref2)[0]
+    assert bad.size == 0, f"E2M1 mismatch at {vals[bad[:8]]}: gpu {e2.cpu().numpy()[bad[:8]]} oracle {ref2[bad[:8]]}"
+    # E4M3 on non-negative inputs: all midpoints +-1 ulp, codes, random
+    table = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    m = ((table[:-1] + table[1:]) / 2).astype(np.float32)
+    pos = np.concatenate([m, np.nextafter(m, np.float32(1e9)), np.nextafter(m, np.float32(0)),
+                          table.astype(np.float32), np.array([448, 464, 465, 1e6, 0, 2.0 ** -10], np.float32),
+                          np.exp(rng.uniform(np.log(1e-5), np.log(600), 1_000_000)).astype(np.float32),
+                          np.abs(f[np.abs(f) < 1e6])]).astype(np.float32)
+    _, e4 = api.debug_encode(torch.from_numpy(pos).to(cuda))
+    ref4 = oracle.e4m3_encode(pos)
+    bad = np.nonzero(e4.cpu().numpy() != ref4)[0]
+    assert bad.size == 0, f"E4M3 mismatch at {pos[bad[:8]]}"
+
+
+def _quant_parity(cuda, x, rac_k, rtol=SCORE_RTOL):
+    M, K = x.shape
+    xd = to_bf16_dev(x, cuda)
+    q = api.quantize(xd, rac_k=rac_k, want_score=True)
+    torch.cuda.synchronize()
+    ref = oracle.quantize(x)
+    assert q.s_t.item() == np.float32(ref.s_t)
+    assert np.array_equal(q.codes.cpu().numpy(), ref.codes)
+    assert np.array_equal(unswizzle(q.scales, M, K), ref.sf)
+    score = oracle.channel_score(ref.resid)
+    np.testing.assert_allclose(q.score.cpu().numpy(), score, rtol=rtol, atol=0)
+    if rac_k:
+        S = oracle.select_topk(score, rac_k)
+        sel = q.sel.cpu().numpy()[:rac_k]
+        check_selection(sel, score, S, rac_k)
+        rho_ref = oracle.rac_residual(ref.resid, ref.s_t, sel)
+        rsel = np_u16(q.r_sel)
+        assert np.array_equal(rsel[:, :rac_k], rho_ref)
+        assert np.all(rsel[:, rac_k:] == 0)
+    return q, ref
+
+
+@pytest.mark.parametrize("M,K,k", [(64, 256, 8), (1, 64, 1), (300, 768, 32), (129, 1536, 64),
+                                   (1000, 2048, 64), (257, 4096, 128), (64, 320, 5), (40, 16384, 256)])
+def test_quantize_parity(cuda, M, K, k):
+    rng = np.random.default_rng(M * 31 + K)
+    _quant_parity(cuda, gen_x(rng, M, K), k)
+
+
+def test_quantize_zero_and_tiny(cuda):
+    x = np.zeros((130, 256), np.uint16)
+    q, ref = _quant_parity(cuda, x, 8)
+    assert q.s_t.item() == 1.0
+    rng = np.random.default_rng(5)
+    y = gen_x(rng, 70, 128, scale=1e-3)
+    y[:, 16:48] = 0
+    y[3, 5] = 0x8000          # -0
+    _quant_parity(cuda, y, 16)
+
+
+def test_quantize_empty(cuda):
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device=cuda)
+    q = api.quantize(x, rac_k=0, m_out=0, want_score=True)
+    torch.cuda.synchronize()
+    assert q.s_t.item() == 1.0 and np.all(q.score.cpu().numpy() == 0)
+
+
+def test_quantize_fanout_and_valid_rows(cuda):
+    """dst_rows fan-out writes every copy; m_valid limits the rows read."""
+    rng = np.random.default_rng(6)
+    M, K, F = 200, 512, 3
+    x = gen_x(rng, M, K)
+    perm = rng.permutation(M * F + 100)[: M * F].astype(np.int32).reshape(M, F)
+    perm[7, 1] = -1
+    m_out = -(-(M * F + 100) // 128) * 128
+    xd = to_bf16_dev(x, cuda)
+    q = api.quantize(xd, rac_k=16, dst_rows=torch.from_numpy(perm).to(cuda), fanout=F, m_out=m_out)
+    torch.cuda.synchronize()
+    ref = oracle.quantize(x)
+    codes = q.codes.cpu().numpy()
+    sf = unswizzle(q.scales, m_out, K)
+    rsel = np_u16(q.r_sel)
+    score = oracle.channel_score(ref.resid)
+    sel = q.sel.cpu().numpy()[:16]
+    check_selection(sel, score, oracle.select_topk(score, 16), 16)
+    rho = oracle.rac_residual(ref.resid, ref.s_t, sel)
+    for r in range(M):
+        for j in range(F):
+            d = perm[r, j]
+            if d < 0:
+                continue
+            assert np.array_equal(codes[d], ref.codes[r])
+            assert np.array_equal(sf[d], ref.sf[r])
+            assert np.array_equal(rsel[d, :16], rho[r])
+    # m_valid: only the first 77 rows count
+    mv = torch.tensor([77], dtype=torch.int32, device=cuda)
+    q2 = api.quantize(xd, rac_k=16, m_valid=mv, want_score=True)
+    torch.cuda.synchronize()
+    ref2 = oracle.quantize(x[:77])
+    assert q2.s_t.item() == np.float32(ref2.s_t)
+    assert np.array_equal(q2.codes.cpu().numpy()[:77], ref2.codes)
+    np.testing.assert_allclose(q2.score.cpu().numpy(), oracle.channel_score(ref2.resid), rtol=SCORE_RTOL)
+
+
+def test_select_ties(cuda):
+    """Equal channel scores: lower channel index first (all-equal columns)."""
+    x = np.tile(gen_x(np.random.default_rng(7), 1, 64), (50, 4))     # K = 256, repeated column groups
+    q, ref = _quant_parity(cuda, x, 10)
+
+
+@pytest.mark.parametrize("G,rows,cols", [(3, 256, 512), (2, 200, 64), (5, 1536, 2048)])
+def test_qdq_weights_parity(cuda, G, rows, cols):
+    rng = np.random.default_rng(G * rows + cols)
+    w = oracle.f32_to_bf16(rng.standard_normal((G, rows, cols)).astype(np.float32) * 0.02)
+    wd = to_bf16_dev(w, cuda)
+    wq, s_t, codes, scales = api.qdq_weights(wd, want_qdq=True, want_packed=True)
+    torch.cuda.synchronize()
+    wq = np_u16(wq)
+    for g in range(G):
+        ref_bf16, ref_s, ref = oracle.qdq(w[g])
+        assert s_t[g].item() == np.float32(ref_s)
+        assert np.array_equal(wq[g], ref_bf16)
+        assert np.array_equal(codes[g].cpu().numpy(), ref.codes)
+        assert np.array_equal(unswizzle(scales[g], rows, cols), ref.sf)
+
+
+@pytest.mark.parametrize("T,E,kr", [(512, 8, 2), (1000, 128, 8), (64, 1, 1), (3, 16, 4), (4096, 256, 8)])
+def test_route_parity(cuda, T, E, kr):
+    rng = np.random.default_rng(T + E)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    if E > 4:
+        logits[0, [1, 3]] = 5.0      # tie
+    r = api.route(torch.from_numpy(logits).to(cuda), kr)
+    torch.cuda.synchronize()
+    idx, gate = oracle.route(logits, kr)
+    assert np.array_equal(r.topk_idx.cpu().numpy(), idx)
+    np.testing.assert_allclose(r.topk_gate.cpu().numpy(), gate, rtol=2e-6, atol=1e-7)
+    off = r.offsets.cpu().numpy()
+    counts = np.bincount(idx.reshape(-1), minlength=E)
+    padded = -(-counts // 128) * 128
+    assert np.array_equal(off, np.concatenate([[0], np.cumsum(padded)]))
+    dst = r.dst_row.cpu().numpy()
+    tok = r.row_token.cpu().numpy()
+    rg = r.row_gate.cpu().numpy()
+    for e in range(E):
+        seg = tok[off[e]:off[e + 1]]
+        toks = np.nonzero((idx == e).any(axis=1))[0]
+        assert np.array_equal(seg[: counts[e]], toks)            # ascending tokens
+        assert np.all(seg[counts[e]:] == -1)
+    assert np.all(tok[off[E]:] == -1)
+    for t in range(T):
+        for j in range(kr):
+            d = dst[t, j]
+            assert tok[d] == t and off[idx[t, j]] <= d < off[idx[t, j] + 1]
+            assert rg[d] == r.topk_gate[t, j].item()
+
+
+def test_gather_weight_channels(cuda):
+    rng = np.random.default_rng(8)
+    E, N, K = 3, 256, 512
+    w = oracle.f32_to_bf16(rng.standard_normal((E, N, K)).astype(np.float32) * 0.02)
+    _, s_t, codes, scales = api.qdq_weights(to_bf16_dev(w, cuda), want_qdq=False, want_packed=True)
+    sel = np.sort(rng.choice(K, 40, replace=False)).astype(np.int32)
+    out = api.gather_weight_channels(codes, scales, N, K, torch.from_numpy(sel).to(cuda), 40, 64)
+    torch.cuda.synchronize()
+    got = np_u16(out)
+    for e in range(E):
+        ref = oracle.quantize(w[e])
+        q = np.empty((N, K), np.uint8)
+        q[:, 0::2] = ref.codes & 0xF
+        q[:, 1::2] = ref.codes >> 4
+        vals = oracle.e2m1_decode(q) * np.repeat(oracle.e4m3_decode(ref.sf), 16, axis=1)
+        want = oracle.f32_to_bf16(vals[:, sel].astype(np.float32))
+        assert np.array_equal(got[e, :, :40], want)
+        assert np.all(got[e, :, 40:] == 0)
