@@ -45,12 +45,13 @@ QUANT_BYTES_PER_ELEM = 2.5625   # 2 B bf16 read + 0.5 B codes + 1/16 B scale wri
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
 
@@ -112,7 +113,7 @@ class ClockSampler:
             try:
                 self.f = open(self.path, "w")
                 self.proc = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.QUERY}",
-                                              "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                              "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
                                              stderr=subprocess.DEVNULL)
             except Exception:
                 self.proc = None
@@ -197,6 +198,8 @@ def run_ours(args):
     import quantization_nvfp4_quantize_b200.moe as moe_mod
     moe_mod.api = api
     clocks = ClockSampler(local, enabled=not args.no_clocks)
+    if clocks.proc is not None:
+        time.sleep(0.5)                 # let the sampler start before the timed region
     torch.cuda.synchronize()
     barrier()
     t0 = torch.cuda.Event(enable_timing=True)
@@ -251,7 +254,7 @@ def run_ours(args):
         "gpu_launches": n_launch_per_step * args.steps,
         "clocks": clk,
     }
-    if rank == 0 and ws == 1:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=8)
     if rank == 0:
         print(json.dumps(out), flush=True)

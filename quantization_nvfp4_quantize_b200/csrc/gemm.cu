@@ -1,7 +1,7 @@
 // gemm.cu -- persistent grouped W4A4 (NVFP4) expert GEMM with Residual
 // Activation Compensation on the sm_100a tensor cores.
 //
-// One CTA per SM, 6 warps:
+// One CTA per SM, 10 warps:
 //   warp 0      TMA producer (one lane): per 256-element K step it loads the
 //               A tile (128 rows x 128 B of packed E2M1), the B tile (two
 //               128-row boxes), and the matching 512-byte scale atoms (bulk
@@ -13,9 +13,12 @@
 //               TMEM accumulator; after the FP4 K loop it drains (commit +
 //               wait) and accumulates the RAC stages with kind::f16 BF16 MMAs
 //               (M128 N256 K16) into the same accumulator.
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, y = s_a s_b D,
-//               then store f32 / SwiGLU -> bf16 / router-weighted atomic
-//               scatter-add into the token-major output.
+//   warps 2..9  epilogue: each warp copies its TMEM slice (32-lane quadrant
+//               w % 4, one half of the columns) into registers and releases
+//               the accumulator at once, so the next tile's MMAs overlap the
+//               math and stores: y = s_a s_b D, then store f32 / SwiGLU ->
+//               bf16 / router-weighted atomic scatter-add into the token-major
+//               output.
 // Tiles: 128 routed rows x 256 output features (SwiGLU: 128 gate + the 128
 // matching up features).  Every expert's routed-row segment is a multiple of
 // 128, so a tile never spans two experts; the tile count comes from the
@@ -45,7 +48,8 @@ constexpr uint32_t SFA_BYTES = 4 * 512;         // 4 atoms (K=256 / 64)
 constexpr uint32_t SFB_BYTES = 8 * 512;         // 2 row blocks x 4 atoms
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr uint32_t RAC_STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;           // producer, MMA, 8 epilogue warps
+constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
 constexpr int MAX_E = 256;
@@ -111,7 +115,7 @@ __device__ __forceinline__ int find_expert(const int *off, int E, int m0)
     return lo;
 }
 
-__device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -131,7 +135,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             ptx::mbar_init(ptx::smem_u32(&sh->empty[s]), 1);
         }
         ptx::mbar_init(ptx::smem_u32(&sh->tmem_full), 1);
-        ptx::mbar_init(ptx::smem_u32(&sh->tmem_empty), 4);
+        ptx::mbar_init(ptx::smem_u32(&sh->tmem_empty), EPI_WARPS);
         ptx::mbar_init(ptx::smem_u32(&sh->drain), 1);
         sh->abort_flag = 0;
         ptx::fence_mbar_init();
@@ -288,7 +292,11 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
         __syncwarp();
     } else {
         // ------------------------------------------------------- epilogue
-        const int q = warp & 3;                 // TMEM lane quadrant of this warp
+        // Warp w owns TMEM lane quadrant w % 4 (32 rows) and one half of the
+        // tile's columns; it copies its whole slice to registers, frees the
+        // accumulator for the next tile's MMAs, then computes and stores.
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int row_in_tile = q * 32 + lane;
         const float s_a = *p.a_s_t;
         int iter = 0;
@@ -301,71 +309,64 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             const int mt = t / n_tiles, nt = t % n_tiles;
             const int m0 = mt * BM;
             const int e = find_expert(sh->offsets, E, m0);
-            const float scale = __fmul_rn(s_a, p.b_s_t[e]);
-            const int64_t r = (int64_t)m0 + row_in_tile;
-            const int token = p.row_token[r];
             const uint32_t tbase = tmem + ACC_COL + ((uint32_t)(q * 32) << 16);
-            if (p.epilogue == MOE_EPI_SWIGLU_BF16) {
-                __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(p.out) + r * p.ld_out + nt * 128;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t g[32], u[32];
-                    ptx::tmem_ld_32x32b_x32(tbase + c * 32, g);
-                    ptx::tmem_ld_32x32b_x32(tbase + 128 + c * 32, u);
-                    ptx::tmem_ld_wait();
-                    uint32_t packed[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        float h0 = 0.0f, h1 = 0.0f;
-                        if (token >= 0) {
-                            float g0 = scale * __uint_as_float(g[2 * j]), u0 = scale * __uint_as_float(u[2 * j]);
-                            float g1 = scale * __uint_as_float(g[2 * j + 1]), u1 = scale * __uint_as_float(u[2 * j + 1]);
-                            h0 = silu(g0) * u0;
-                            h1 = silu(g1) * u1;
-                        }
-                        packed[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h0)) |
-                                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h1)) << 16);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + c * 32);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-                }
-            } else if (p.epilogue == MOE_EPI_STORE_F32) {
-                float *out = reinterpret_cast<float *>(p.out) + r * p.ld_out + nt * BN;
-#pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t v[32];
-                    ptx::tmem_ld_32x32b_x32(tbase + c * 32, v);
-                    ptx::tmem_ld_wait();
-                    if (token >= 0) {
-                        float4 *dst = reinterpret_cast<float4 *>(out + c * 32);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            dst[j] = make_float4(scale * __uint_as_float(v[4 * j]), scale * __uint_as_float(v[4 * j + 1]),
-                                                 scale * __uint_as_float(v[4 * j + 2]), scale * __uint_as_float(v[4 * j + 3]));
-                    }
-                }
+            uint32_t v[128];
+            if (swiglu) {
+                // gate columns [64 half, +64) and the matching up columns
+                ptx::tmem_ld_32x32b_x32(tbase + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                ptx::tmem_ld_32x32b_x32(tbase + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                ptx::tmem_ld_32x32b_x32(tbase + 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
+                ptx::tmem_ld_32x32b_x32(tbase + 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
             } else {
-                const float gw = token >= 0 ? __fmul_rn(scale, p.row_gate[r]) : 0.0f;
-                float *out = reinterpret_cast<float *>(p.out) + (int64_t)(token >= 0 ? token : 0) * p.ld_out + nt * BN;
-#pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t v[32];
-                    ptx::tmem_ld_32x32b_x32(tbase + c * 32, v);
-                    ptx::tmem_ld_wait();
-                    if (token >= 0) {
-                        float4 *dst = reinterpret_cast<float4 *>(out + c * 32);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            atomicAdd(dst + j, make_float4(gw * __uint_as_float(v[4 * j]), gw * __uint_as_float(v[4 * j + 1]),
-                                                           gw * __uint_as_float(v[4 * j + 2]), gw * __uint_as_float(v[4 * j + 3])));
-                    }
-                }
+                for (int c = 0; c < 4; ++c)
+                    ptx::tmem_ld_32x32b_x32(tbase + half * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
             }
+            ptx::tmem_ld_wait();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&sh->tmem_empty));
+
+            const float scale = __fmul_rn(s_a, p.b_s_t[e]);
+            const int64_t r = (int64_t)m0 + row_in_tile;
+            const int token = p.row_token[r];
+            if (p.epilogue == MOE_EPI_SWIGLU_BF16) {
+                uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + r * p.ld_out +
+                                                       nt * 128 + half * 64);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = c * 8 + jj * 2;
+                        float h0 = 0.0f, h1 = 0.0f;
+                        if (token >= 0) {
+                            h0 = silu(scale * __uint_as_float(v[j])) * (scale * __uint_as_float(v[64 + j]));
+                            h1 = silu(scale * __uint_as_float(v[j + 1])) * (scale * __uint_as_float(v[64 + j + 1]));
+                        }
+                        w4[jj] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h0)) |
+                                 ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h1)) << 16);
+                    }
+                    dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            } else if (p.epilogue == MOE_EPI_STORE_F32) {
+                if (token >= 0) {
+                    float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + r * p.ld_out +
+                                                             nt * BN + half * 128);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        dst[j] = make_float4(scale * __uint_as_float(v[4 * j]), scale * __uint_as_float(v[4 * j + 1]),
+                                             scale * __uint_as_float(v[4 * j + 2]), scale * __uint_as_float(v[4 * j + 3]));
+                }
+            } else if (token >= 0) {
+                const float gw = __fmul_rn(scale, p.row_gate[r]);
+                float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + (int64_t)token * p.ld_out +
+                                                         nt * BN + half * 128);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    atomicAdd(dst + j, make_float4(gw * __uint_as_float(v[4 * j]), gw * __uint_as_float(v[4 * j + 1]),
+                                                   gw * __uint_as_float(v[4 * j + 2]), gw * __uint_as_float(v[4 * j + 3])));
+            }
         }
     }
 

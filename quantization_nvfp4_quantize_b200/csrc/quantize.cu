@@ -15,7 +15,8 @@
 // one range of rows.  Each lane owns 8 consecutive channels (one 16-byte
 // load), two lanes form a 16-element block (amax by one xor-shuffle), a warp
 // reads 512 contiguous bytes of a row.  Lanes keep their channels' residual
-// sums across rows (binary32 for 4 rows, then binary64), the CTA reduces its
+// sums across rows (binary32 for up to 4 rows, then binary64; each warp keeps
+// 4 rows' loads in flight), the CTA reduces its
 // 8 warps in shared memory and writes one partial per channel; partials are
 // summed in a fixed order by k_score_reduce, so scores are deterministic.
 #include "common.cuh"
@@ -26,7 +27,8 @@ namespace nvfp4 {
 
 constexpr int QTHREADS = 256;
 constexpr int QCHUNK = 256;           // channels per CTA column chunk
-constexpr int SCORE_FLUSH = 4;        // rows summed in binary32 before binary64
+constexpr int ROWS_IN_FLIGHT = 4;     // rows a warp loads before processing them; also the
+                                      // number of rows summed in binary32 before binary64
 
 // -------------------------------------------------------------------- amax
 
@@ -112,68 +114,75 @@ __global__ void __launch_bounds__(QTHREADS) k_quantize(QuantParams p)
     double acc64[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) { acc32[i] = 0.0f; acc64[i] = 0.0; }
-    int since_flush = 0;
 
     const int64_t kb0 = c >> 4;                 // first block of the 4-block group (lanes 8j)
-    for (int64_t r = r0 + warp; r < r1; r += QTHREADS / 32) {
-        float v[8];
-        if (active) {
-            uint4 u = __ldg(reinterpret_cast<const uint4 *>(xg + r * p.ldx + c));
-            v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-            v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
-        } else {
+    constexpr int WARPS = QTHREADS / 32;
+    for (int64_t rbase = r0 + warp; rbase < r1; rbase += ROWS_IN_FLIGHT * WARPS) {
+        // issue every row's load first: ROWS_IN_FLIGHT 16-byte loads per lane in flight
+        uint4 u[ROWS_IN_FLIGHT];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+        for (int i = 0; i < ROWS_IN_FLIGHT; ++i) {
+            const int64_t r = rbase + (int64_t)i * WARPS;
+            u[i] = (active && r < r1) ? __ldg(reinterpret_cast<const uint4 *>(xg + r * p.ldx + c))
+                                      : make_uint4(0u, 0u, 0u, 0u);
         }
-        float m = fabsf(v[0]);
 #pragma unroll
-        for (int i = 1; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        BlockScale bs = block_scale(m, s_t, r6);
-        float xh[8];
-        uint32_t cw = quant8(v, bs, xh);
+        for (int i = 0; i < ROWS_IN_FLIGHT; ++i) {
+            const int64_t r = rbase + (int64_t)i * WARPS;
+            if (r >= r1) break;                 // warp-uniform
+            float v[8];
+            v[0] = bf16lo(u[i].x); v[1] = bf16hi(u[i].x); v[2] = bf16lo(u[i].y); v[3] = bf16hi(u[i].y);
+            v[4] = bf16lo(u[i].z); v[5] = bf16hi(u[i].z); v[6] = bf16lo(u[i].w); v[7] = bf16hi(u[i].w);
+            float m = fabsf(v[0]);
+#pragma unroll
+            for (int k = 1; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            BlockScale bs = block_scale(m, s_t, r6);
+            float xh[8];
+            uint32_t cw = quant8(v, bs, xh);
 
-        // gather the 4 scale codes of blocks kb0..kb0+3 onto lanes 8j
-        uint32_t s1 = __shfl_down_sync(0xffffffffu, bs.sf_code, 2);
-        uint32_t s2 = __shfl_down_sync(0xffffffffu, bs.sf_code, 4);
-        uint32_t s3 = __shfl_down_sync(0xffffffffu, bs.sf_code, 6);
-        uint32_t sw = bs.sf_code | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            // gather the 4 scale codes of blocks kb0..kb0+3 onto lanes 8j
+            uint32_t s1 = __shfl_down_sync(0xffffffffu, bs.sf_code, 2);
+            uint32_t s2 = __shfl_down_sync(0xffffffffu, bs.sf_code, 4);
+            uint32_t s3 = __shfl_down_sync(0xffffffffu, bs.sf_code, 6);
+            uint32_t sw = bs.sf_code | (s1 << 8) | (s2 << 16) | (s3 << 24);
 
-        if (active) {
-            if (SCORE) {
+            if (active) {
+                if (SCORE) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float R = __fsub_rn(v[i], xh[i]);
-                    acc32[i] = fmaf(R, R, acc32[i]);
+                    for (int k = 0; k < 8; ++k) {
+                        float R = __fsub_rn(v[k], xh[k]);
+                        acc32[k] = fmaf(R, R, acc32[k]);
+                    }
                 }
-                if (++since_flush == SCORE_FLUSH) {
+                if (qdq) {
+                    uint4 o;
+                    o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[0])) |
+                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[1])) << 16);
+                    o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[2])) |
+                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[3])) << 16);
+                    o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[4])) |
+                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[5])) << 16);
+                    o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[6])) |
+                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[7])) << 16);
+                    *reinterpret_cast<uint4 *>(qdq + r * K + c) = o;
+                }
+                if (codes) {
+                    const int nd = p.dst_rows ? p.fanout : 1;
+                    for (int j = 0; j < nd; ++j) {
+                        int64_t dst = p.dst_rows ? (int64_t)p.dst_rows[r * p.fanout + j] : r;
+                        if (dst < 0) continue;
+                        *reinterpret_cast<uint32_t *>(codes + dst * (K >> 1) + (c >> 1)) = cw;
+                        if ((lane & 7) == 0)
+                            *reinterpret_cast<uint32_t *>(scales + sf_offset(dst, kb0, K)) = sw;
+                    }
+                }
+            }
+        }
+        if (SCORE) {
+            // at most ROWS_IN_FLIGHT rows were summed in binary32
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) { acc64[i] += (double)acc32[i]; acc32[i] = 0.0f; }
-                    since_flush = 0;
-                }
-            }
-            if (qdq) {
-                uint4 o;
-                o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[0])) |
-                      ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[1])) << 16);
-                o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[2])) |
-                      ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[3])) << 16);
-                o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[4])) |
-                      ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[5])) << 16);
-                o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[6])) |
-                      ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[7])) << 16);
-                *reinterpret_cast<uint4 *>(qdq + r * K + c) = o;
-            }
-            if (codes) {
-                const int nd = p.dst_rows ? p.fanout : 1;
-                for (int j = 0; j < nd; ++j) {
-                    int64_t dst = p.dst_rows ? (int64_t)p.dst_rows[r * p.fanout + j] : r;
-                    if (dst < 0) continue;
-                    *reinterpret_cast<uint32_t *>(codes + dst * (K >> 1) + (c >> 1)) = cw;
-                    if ((lane & 7) == 0)
-                        *reinterpret_cast<uint32_t *>(scales + sf_offset(dst, kb0, K)) = sw;
-                }
-            }
+            for (int k = 0; k < 8; ++k) { acc64[k] += (double)acc32[k]; acc32[k] = 0.0f; }
         }
     }
 
@@ -604,3 +613,4 @@ extern "C" nvfp4_status nvfp4_debug_encode(const float *in_dev, int64_t n, uint8
     k_debug_encode<<<blocks, 256, 0, (cudaStream_t)stream>>>(in_dev, n, e2m1_dev, e4m3_dev);
     return check_launch("k_debug_encode");
 }
+
