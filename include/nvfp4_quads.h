@@ -138,6 +138,42 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, i
                             void *stream);
 
 /* --------------------------------------------------------------------------
+ * nvfp4_quantize_noalloc -- nvfp4_quantize without a caller workspace.  The
+ * QUADS pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory at the moment they quantize: a plug-in
+ * running inside a host framework that owns every device allocation and gives
+ * it no allocator, or a serving loop that reserved all free device memory up
+ * front and may not call cudaMalloc (or wait on its implicit synchronization)
+ * per request.  Such a caller still passes its inputs and outputs; only the
+ * scratch memory moves into the library.
+ *
+ * Arguments, outputs and errors are those of nvfp4_quantize minus
+ * workspace/workspace_bytes.  Scratch is a fixed 4 MiB array in the library's
+ * device memory (nvfp4_quantize_noalloc_max_scratch() returns its size), held
+ * by every GPU that loads the library until the process exits.  Shapes whose
+ * nvfp4_quantize_workspace_size(M, K) exceeds it are rejected with
+ * NVFP4_ERR_UNSUPPORTED_SHAPE.  The call allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents; the call clears what must start at zero itself.  Calls whose
+ *     executions overlap on the GPU (different streams, or several host
+ *     threads) race on the array and give undefined results: serialize them.
+ * -------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_quantize_noalloc_max_scratch(void);
+
+NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
+                                              const int32_t *m_valid_dev,
+                                              const float *s_t_in_dev, float *s_t_out_dev,
+                                              const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
+                                              uint8_t *codes_dev, uint8_t *scales_dev,
+                                              double *score_dev, int32_t rac_k, int32_t rac_ld,
+                                              int32_t *sel_dev, void *r_sel_dev,
+                                              int32_t *dev_status, void *stream);
+
+/* --------------------------------------------------------------------------
  * nvfp4_qdq_weights -- trainer-side asymmetric QAT weight fake-quantization
  * (gist.science/it 2.2 A: weights are quantized to NVFP4 and dequantized on
  * every trainer forward so the trainer sees the rollout's weights; activations

@@ -25,6 +25,10 @@ SIGNATURES = {
     "nvfp4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_int32, c_int64, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "nvfp4_quantize_noalloc_max_scratch": (c_size_t, []),
+    "nvfp4_quantize_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+                                         c_void_p, c_int32, c_int64, c_void_p, c_void_p, c_void_p, c_int32,
+                                         c_int32, c_void_p, c_void_p, c_void_p, c_void_p]),
     "nvfp4_qdq_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
     "nvfp4_qdq_weights": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
                                     c_void_p, c_void_p, c_size_t, c_void_p]),

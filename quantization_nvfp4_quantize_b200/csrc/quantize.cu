@@ -22,6 +22,7 @@
 #include "common.cuh"
 
 #include <algorithm>
+#include <mutex>
 
 namespace nvfp4 {
 
@@ -614,3 +615,70 @@ extern "C" nvfp4_status nvfp4_debug_encode(const float *in_dev, int64_t n, uint8
     return check_launch("k_debug_encode");
 }
 
+// ------------------------------------------------- allocation-free variant
+//
+// nvfp4_quantize_noalloc serves callers that cannot allocate device memory
+// when they call in (see the header).  Its scratch space -- the amax slot and
+// the per-CTA score partials that nvfp4_quantize keeps in the caller's
+// workspace -- lives in this file-scope device array instead, which every
+// GPU that loads the library holds until the process exits.  In host code
+// the array's name is only a host-side stand-in, so its device address is
+// looked up once per device with cudaGetSymbolAddress (on the first call made
+// with that device current) and passed to the kernels.
+
+namespace nvfp4 {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(4) << 20;     // 4 MiB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+static void *noalloc_scratch_ptr(nvfp4_status *st)
+{
+    static void *ptrs[64];
+    static std::mutex mu;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        *st = set_error(NVFP4_ERR_CUDA, "nvfp4_quantize_noalloc: no usable current device");
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            *st = set_error(NVFP4_ERR_CUDA, "nvfp4_quantize_noalloc: cudaGetSymbolAddress failed: %s",
+                            cudaGetErrorString(e));
+            return nullptr;
+        }
+        ptrs[dev] = p;
+    }
+    *st = NVFP4_OK;
+    return ptrs[dev];
+}
+
+}  // namespace nvfp4
+
+extern "C" size_t nvfp4_quantize_noalloc_max_scratch(void) { return nvfp4::NOALLOC_SCRATCH_BYTES; }
+
+extern "C" nvfp4_status nvfp4_quantize_noalloc(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
+                                               const int32_t *m_valid_dev,
+                                               const float *s_t_in_dev, float *s_t_out_dev,
+                                               const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
+                                               uint8_t *codes_dev, uint8_t *scales_dev,
+                                               double *score_dev, int32_t rac_k, int32_t rac_ld,
+                                               int32_t *sel_dev, void *r_sel_dev,
+                                               int32_t *dev_status, void *stream)
+{
+    size_t need = nvfp4_quantize_workspace_size(M, K);
+    NVFP4_REQUIRE(need > 0, NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_noalloc: bad sizes");
+    NVFP4_REQUIRE(need <= nvfp4::NOALLOC_SCRATCH_BYTES, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_quantize_noalloc: M=%lld, K=%lld needs %zu bytes of scratch, above the fixed %zu-byte "
+                  "device array; call nvfp4_quantize with a workspace instead",
+                  (long long)M, (long long)K, need, nvfp4::NOALLOC_SCRATCH_BYTES);
+    nvfp4_status st;
+    void *scratch = nvfp4::noalloc_scratch_ptr(&st);
+    if (!scratch) return st;
+    return nvfp4_quantize(x_dev, M, K, ldx, m_valid_dev, s_t_in_dev, s_t_out_dev, dst_rows_dev, fanout, M_out,
+                          codes_dev, scales_dev, score_dev, rac_k, rac_ld, sel_dev, r_sel_dev, dev_status, scratch,
+                          nvfp4::NOALLOC_SCRATCH_BYTES, stream);
+}
