@@ -236,6 +236,30 @@ NVFP4_API nvfp4_status nvfp4_gather_weight_channels(const uint8_t *codes_dev, co
                                           void *w_sel_dev, void *stream);
 
 /* --------------------------------------------------------------------------
+ * nvfp4_weights_channel_major -- one-time channel-major copy of E NVFP4
+ * weights [N x K] (made when weights are loaded; they do not change between
+ * steps) so that the per-step RAC weight gather reads only the selected
+ * channels:
+ *   codes_cm_dev  uint8 [E x K x N/2]: row c holds the codes of input
+ *                 channel c for all N output features (even n in the low
+ *                 nibble).
+ *   scales_cm_dev uint8 [E x K/16 x N]: row b holds the E4M3 scale of block
+ *                 b of every output feature.
+ * N % 64 == 0, K % 64 == 0.
+ *
+ * nvfp4_gather_weight_channels_cm -- nvfp4_gather_weight_channels from the
+ * channel-major copy (identical output: w_sel[e, n, j] = bf16(e2m1 * sf) of
+ * channel S_j, zero for k <= j < ld).
+ * -------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_weights_channel_major(const uint8_t *codes_dev, const uint8_t *scales_dev, int32_t E,
+                                                   int64_t N, int64_t K, uint8_t *codes_cm_dev,
+                                                   uint8_t *scales_cm_dev, void *stream);
+
+NVFP4_API nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_dev, const uint8_t *scales_cm_dev,
+                                                       int32_t E, int64_t N, int64_t K, const int32_t *sel_dev,
+                                                       int32_t k, int32_t ld, void *w_sel_dev, void *stream);
+
+/* --------------------------------------------------------------------------
  * moe_w4a4_grouped_gemm_rac -- the native W4A4 block-scaled grouped expert
  * GEMM with Residual Activation Compensation folded into the same
  * accumulator (gist.science/it 2.2 B; shd-paper.top abstract: RAC corrects

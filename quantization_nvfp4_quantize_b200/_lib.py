@@ -37,6 +37,10 @@ SIGNATURES = {
                             c_void_p, c_void_p, c_int64, c_void_p, c_size_t, c_void_p]),
     "nvfp4_gather_weight_channels": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int64, c_void_p,
                                                c_int32, c_int32, c_void_p, c_void_p]),
+    "nvfp4_weights_channel_major": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int64, c_void_p, c_void_p,
+                                              c_void_p]),
+    "nvfp4_gather_weight_channels_cm": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int64, c_void_p,
+                                                  c_int32, c_int32, c_void_p, c_void_p]),
     "moe_w4a4_grouped_gemm_rac": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
                                             c_void_p, c_int64, c_int64, c_int32, c_void_p, c_int32, c_void_p,
                                             c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_void_p,

@@ -147,6 +147,27 @@ def gather_weight_channels(codes: torch.Tensor, scales: torch.Tensor, N: int, K:
     return out
 
 
+def weights_channel_major(codes: torch.Tensor, scales: torch.Tensor, N: int, K: int):
+    """nvfp4_weights_channel_major: (codes_cm [E, K, N/2], scales_cm [E, K/16, N])."""
+    lib = _lib.load()
+    E = codes.shape[0]
+    ccm = torch.empty(E, K, N // 2, dtype=U8, device=codes.device)
+    scm = torch.empty(E, K // 16, N, dtype=U8, device=codes.device)
+    check(lib.nvfp4_weights_channel_major(_p(codes), _p(scales), E, N, K, _p(ccm), _p(scm), _stream(codes.device)))
+    return ccm, scm
+
+
+def gather_weight_channels_cm(codes_cm: torch.Tensor, scales_cm: torch.Tensor, N: int, K: int, sel: torch.Tensor,
+                              k: int, ld: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    lib = _lib.load()
+    E = codes_cm.shape[0]
+    if out is None:
+        out = torch.empty(E, N, ld, dtype=BF16, device=codes_cm.device)
+    check(lib.nvfp4_gather_weight_channels_cm(_p(codes_cm), _p(scales_cm), E, N, K, _p(sel), k, ld, _p(out),
+                                              _stream(codes_cm.device)))
+    return out
+
+
 def grouped_gemm(a_codes, a_scales, a_s_t, m_pad_max, b_codes, b_scales, b_s_t, N, K, E, offsets, *,
                  rac_ld=0, rho=None, w_sel=None, epilogue=EPI_STORE_F32, row_token=None, row_gate=None,
                  out=None, ld_out=None, dev_status=None):

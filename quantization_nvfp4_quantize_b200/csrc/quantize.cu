@@ -28,6 +28,7 @@ namespace nvfp4 {
 
 constexpr int QTHREADS = 256;
 constexpr int QCHUNK = 256;           // channels per CTA column chunk
+constexpr int QCTAS_PER_SM = 4;       // resident CTAs per SM the grid is sized for (one wave)
 constexpr int ROWS_IN_FLIGHT = 4;     // rows a warp loads before processing them; also the
                                       // number of rows summed in binary32 before binary64
 
@@ -89,7 +90,7 @@ struct QuantParams {
 };
 
 template <bool SCORE>
-__global__ void __launch_bounds__(QTHREADS) k_quantize(QuantParams p)
+__global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(QuantParams p)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = blockIdx.z;
@@ -271,16 +272,30 @@ __global__ void __launch_bounds__(1024) k_select_topk(const double *__restrict__
             if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255ull], 1u);
         }
         __syncthreads();
-        if (tid == 0) {
-            int rem = s_rem;
-            unsigned int above = 0;
-            int d = 255;
-            for (; d > 0; --d) {
-                if (above + hist[d] >= (unsigned)rem) break;
-                above += hist[d];
+        if (tid < 32) {
+            // warp 0 finds the digit: lane l owns bins 255-8l .. 248-8l (descending)
+            const int rem = s_rem;
+            unsigned int cnt[8], tot = 0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) { cnt[b] = hist[255 - 8 * tid - b]; tot += cnt[b]; }
+            unsigned int incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                unsigned int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (tid >= o) incl += v;
             }
-            s_digit = d;
-            s_rem = rem - (int)above;
+            unsigned int above = incl - tot;          // keys in higher bins than this lane's
+            bool mine = above < (unsigned)rem && (unsigned)rem <= incl;
+            if (mine) {
+                unsigned int a = above;
+                int b = 0;
+                for (; b < 7; ++b) {
+                    if (a + cnt[b] >= (unsigned)rem) break;
+                    a += cnt[b];
+                }
+                s_digit = 255 - 8 * tid - b;
+                s_rem = rem - (int)a;
+            }
         }
         __syncthreads();
         prefix |= (unsigned long long)s_digit << shift;
@@ -388,12 +403,85 @@ __global__ void k_gather_w_channels(const uint8_t *__restrict__ codes, const uin
     }
 }
 
+// ------------------------------------------- channel-major weight copies
+
+// codes_cm[e][c][n/2] (element (n, c), even n in the low nibble) and
+// scales_cm[e][c/16][n] from the K-major NVFP4 weight.  One thread per output
+// code byte; the scale row is written by the threads whose c % 16 == 0.
+__global__ void k_weights_channel_major(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                                        int64_t E, int64_t N, int64_t K, uint8_t *__restrict__ codes_cm,
+                                        uint8_t *__restrict__ scales_cm)
+{
+    const int64_t total = E * K * (N / 2);
+    const int64_t sf_per_e = sf_bytes(N, K);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t np = i % (N / 2);           // pair of n
+        const int64_t ec = i / (N / 2);
+        const int64_t c = ec % K, e = ec / K;
+        const int64_t n0 = 2 * np;
+        const uint8_t *row0 = codes + (e * N + n0) * (K / 2);
+        const uint8_t *row1 = row0 + K / 2;
+        uint32_t b0 = row0[c >> 1], b1 = row1[c >> 1];
+        uint32_t q0 = (c & 1) ? (b0 >> 4) : (b0 & 15u);
+        uint32_t q1 = (c & 1) ? (b1 >> 4) : (b1 & 15u);
+        codes_cm[i] = (uint8_t)(q0 | (q1 << 4));
+        if ((c & 15) == 0) {
+            const uint8_t *se = scales + e * sf_per_e;
+            uint8_t *dst = scales_cm + (e * (K / 16) + (c >> 4)) * N + n0;
+            dst[0] = se[sf_offset(n0, c >> 4, K)];
+            dst[1] = se[sf_offset(n0 + 1, c >> 4, K)];
+        }
+    }
+}
+
+// RAC weight operand from the channel-major copy: one CTA per (expert, 64
+// output features).  Each selected channel's 64 codes (32 bytes) and scales
+// (64 bytes) are read as contiguous runs, dequantized (e2m1 * sf, exact in
+// bf16) into a shared [channel][feature] tile, then written out transposed as
+// [feature][ld] rows.
+constexpr int GCM_N = 64;
+constexpr int GCM_TS = GCM_N + 1;                     // padded row of the shared tile (floats)
+
+__global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__restrict__ codes_cm,
+                                                              const uint8_t *__restrict__ scales_cm, int64_t N,
+                                                              int64_t K, const int32_t *__restrict__ sel, int k,
+                                                              int ld, __nv_bfloat16 *__restrict__ out)
+{
+    extern __shared__ float gtile[];                   // [ld][GCM_TS]
+    const int64_t e = blockIdx.y;
+    const int64_t n0 = (int64_t)blockIdx.x * GCM_N;
+    // phase 1: thread (j, f) dequantizes feature n0 + f of selected channel j
+    for (int idx = threadIdx.x; idx < ld * GCM_N; idx += blockDim.x) {
+        const int jj = idx / GCM_N;
+        const int f = idx - jj * GCM_N;
+        float v = 0.0f;
+        if (jj < k) {
+            const int64_t ch = sel[jj];
+            const int64_t n = n0 + f;
+            const uint32_t byte = codes_cm[(e * K + ch) * (N / 2) + (n >> 1)];
+            const uint32_t nib = (n & 1) ? (byte >> 4) : (byte & 15u);
+            const float q = e2m1x2_to_f32(nib).x;
+            const float sf = e4m3_to_f32(scales_cm[(e * (K / 16) + (ch >> 4)) * N + n]);
+            v = __fmul_rn(q, sf);
+        }
+        gtile[jj * GCM_TS + f] = v;
+    }
+    __syncthreads();
+    // phase 2: thread (f, j) writes out[e, n0 + f, j]; consecutive threads take consecutive j
+    for (int idx = threadIdx.x; idx < GCM_N * ld; idx += blockDim.x) {
+        const int f = idx / ld;
+        const int jj = idx - f * ld;
+        out[(e * N + n0 + f) * ld + jj] = __float2bfloat16_rn(gtile[jj * GCM_TS + f]);
+    }
+}
+
 // --------------------------------------------------------------- helpers
 
 static int64_t pick_rows_per_cta(int64_t M, int64_t nchunks, int64_t groups)
 {
-    // aim for ~4 CTAs per SM over the whole grid, at least 8 rows per CTA
-    int64_t target = (int64_t)num_sms() * 4;
+    // one full wave: QCTAS_PER_SM resident CTAs per SM, at least 8 rows per CTA
+    int64_t target = (int64_t)num_sms() * QCTAS_PER_SM;
     int64_t per_group = std::max<int64_t>(1, target / std::max<int64_t>(1, nchunks * groups));
     int64_t rpc = (M + per_group - 1) / per_group;
     rpc = std::max<int64_t>(rpc, 8);
@@ -496,10 +584,14 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
     }
     if (rac_k > 0) {
         size_t smem = (size_t)K * sizeof(unsigned long long);
-        static bool attr_set = false;
-        if (!attr_set) {
-            cudaFuncSetAttribute(k_select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, 16384 * 8);
-            attr_set = true;
+        static bool attr_set[64];
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+            if (cudaFuncSetAttribute(k_select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, 16384 * 8) !=
+                cudaSuccess)
+                return check_launch("nvfp4_quantize: smem attribute");
+            attr_set[dev] = true;
         }
         k_select_topk<<<1, 1024, smem, st>>>(score, (int)K, rac_k, sel_dev);
         if (check_launch("k_select_topk") != NVFP4_OK) return NVFP4_ERR_CUDA;
@@ -589,6 +681,50 @@ extern "C" nvfp4_status nvfp4_gather_weight_channels(const uint8_t *codes_dev, c
     k_gather_w_channels<<<blocks, 256, 0, st>>>(codes_dev, scales_dev, E, N, K, sel_dev, k, ld,
                                                 (__nv_bfloat16 *)w_sel_dev);
     return check_launch("k_gather_w_channels");
+}
+
+extern "C" nvfp4_status nvfp4_weights_channel_major(const uint8_t *codes_dev, const uint8_t *scales_dev, int32_t E,
+                                                    int64_t N, int64_t K, uint8_t *codes_cm_dev,
+                                                    uint8_t *scales_cm_dev, void *stream)
+{
+    NVFP4_REQUIRE(codes_dev && scales_dev && codes_cm_dev && scales_cm_dev, NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_weights_channel_major: null pointer");
+    NVFP4_REQUIRE(E >= 1 && N >= 2 && N % 64 == 0 && K >= 64 && K % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_weights_channel_major: need N % 64 == 0, K % 64 == 0");
+    int64_t total = (int64_t)E * K * (N / 2);
+    int blocks = (int)std::min<int64_t>((int64_t)num_sms() * 16, (total + 255) / 256);
+    k_weights_channel_major<<<blocks, 256, 0, (cudaStream_t)stream>>>(codes_dev, scales_dev, E, N, K, codes_cm_dev,
+                                                                     scales_cm_dev);
+    return check_launch("k_weights_channel_major");
+}
+
+extern "C" nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_dev, const uint8_t *scales_cm_dev,
+                                                        int32_t E, int64_t N, int64_t K, const int32_t *sel_dev,
+                                                        int32_t k, int32_t ld, void *w_sel_dev, void *stream)
+{
+    NVFP4_REQUIRE(codes_cm_dev && scales_cm_dev && w_sel_dev && (k == 0 || sel_dev), NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_gather_weight_channels_cm: null pointer");
+    NVFP4_REQUIRE(E >= 1 && E <= 65535 && N >= 64 && N % 64 == 0 && K >= 64 && K % 64 == 0,
+                  NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_gather_weight_channels_cm: need N % 64 == 0, K % 64 == 0");
+    NVFP4_REQUIRE(k >= 0 && k <= ld && ld % 64 == 0 && ld <= 256 && k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_gather_weight_channels_cm: need 0 <= k <= ld <= 256, ld % 64 == 0");
+    NVFP4_REQUIRE(aligned16(w_sel_dev), NVFP4_ERR_ALIGNMENT, "nvfp4_gather_weight_channels_cm: w_sel alignment");
+    size_t smem = (size_t)ld * GCM_TS * sizeof(float);
+    {
+        static bool attr_done[64];
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+            if (cudaFuncSetAttribute(k_gather_w_channels_cm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(256 * GCM_TS * sizeof(float))) != cudaSuccess)
+                return check_launch("nvfp4_gather_weight_channels_cm: smem attribute");
+            attr_done[dev] = true;
+        }
+    }
+    dim3 grid((unsigned)(N / GCM_N), (unsigned)E);
+    k_gather_w_channels_cm<<<grid, 256, smem, (cudaStream_t)stream>>>(codes_cm_dev, scales_cm_dev, N, K, sel_dev, k,
+                                                                    ld, (__nv_bfloat16 *)w_sel_dev);
+    return check_launch("k_gather_w_channels_cm");
 }
 
 // ------------------------------------------------------- conversion probe

@@ -7,10 +7,11 @@ and 2.2 B; shd-paper.top abstract):
   2. nvfp4_quantize(X)         amax -> s_x, codes/scales written to every routed
                                row of each token, channel scores, top-k S_x,
                                RAC residual rho_x for every routed row
-  3. gather_weight_channels    W13q[:, :, S_x] as bf16 (e2m1 * sf)
+  3. gather_weight_channels_cm W13q[:, :, S_x] as bf16 (e2m1 * sf), read from
+                               the channel-major weight copy
   4. grouped GEMM (gate/up)    W4A4 + RAC, epilogue SwiGLU -> h bf16
   5. nvfp4_quantize(h)         over the valid routed rows: s_h, codes, S_h, rho_h
-  6. gather_weight_channels    W2q[:, :, S_h]
+  6. gather_weight_channels_cm W2q[:, :, S_h]
   7. grouped GEMM (down)       W4A4 + RAC, epilogue router-weighted scatter-add
                                into Y [T x H] fp32
 
@@ -37,6 +38,9 @@ class MoELayerW4A4:
         self.rac_ld = -(-rac_k // 64) * 64 if rac_k else 0
         _, self.s13, self.c13, self.sf13 = api.qdq_weights(w13, want_qdq=False, want_packed=True)
         _, self.s2, self.c2, self.sf2 = api.qdq_weights(w2, want_qdq=False, want_packed=True)
+        # channel-major copies: the per-step RAC gathers read only the selected channels
+        self.c13_cm, self.sf13_cm = api.weights_channel_major(self.c13, self.sf13, 2 * I, H)
+        self.c2_cm, self.sf2_cm = api.weights_channel_major(self.c2, self.sf2, H, I)
         self.m_pad = api.padded_rows_bound(tokens, topk, E)
         mp, ld = self.m_pad, max(self.rac_ld, 1)
         self.xq = api.Quantized(
@@ -69,7 +73,8 @@ class MoELayerW4A4:
         api.quantize(x, rac_k=k, rac_ld=self.rac_ld, dst_rows=r.dst_row, fanout=self.k_r, m_out=self.m_pad,
                      out=self.xq, workspace=self.ws_x)
         if k:
-            api.gather_weight_channels(self.c13, self.sf13, 2 * I, H, self.xq.sel, k, self.rac_ld, out=self.w_sel13)
+            api.gather_weight_channels_cm(self.c13_cm, self.sf13_cm, 2 * I, H, self.xq.sel, k, self.rac_ld,
+                                          out=self.w_sel13)
         api.grouped_gemm(self.xq.codes, self.xq.scales, self.xq.s_t, self.m_pad, self.c13, self.sf13, self.s13,
                          2 * I, H, E, r.offsets, rac_ld=self.rac_ld if k else 0, rho=self.xq.r_sel,
                          w_sel=self.w_sel13, epilogue=api.EPI_SWIGLU_BF16, row_token=r.row_token,
@@ -77,7 +82,8 @@ class MoELayerW4A4:
         api.quantize(self.h, rac_k=k, rac_ld=self.rac_ld, m_out=self.m_pad, m_valid=r.offsets[E:],
                      out=self.hq, workspace=self.ws_h)
         if k:
-            api.gather_weight_channels(self.c2, self.sf2, H, I, self.hq.sel, k, self.rac_ld, out=self.w_sel2)
+            api.gather_weight_channels_cm(self.c2_cm, self.sf2_cm, H, I, self.hq.sel, k, self.rac_ld,
+                                          out=self.w_sel2)
         self.y.zero_()
         api.grouped_gemm(self.hq.codes, self.hq.scales, self.hq.s_t, self.m_pad, self.c2, self.sf2, self.s2,
                          H, I, E, r.offsets, rac_ld=self.rac_ld if k else 0, rho=self.hq.r_sel, w_sel=self.w_sel2,

@@ -206,3 +206,31 @@ def test_gather_weight_channels(cuda):
         want = oracle.f32_to_bf16(vals[:, sel].astype(np.float32))
         assert np.array_equal(got[e, :, :40], want)
         assert np.all(got[e, :, 40:] == 0)
+
+
+@pytest.mark.parametrize("E,N,K,k,ld", [(3, 256, 512, 40, 64), (2, 1536, 768, 128, 128), (4, 128, 2048, 256, 256)])
+def test_channel_major_copy_and_gather(cuda, E, N, K, k, ld):
+    """The channel-major weight copy holds the same codes/scales, and the
+    gather from it equals the gather from the K-major weight and the oracle."""
+    rng = np.random.default_rng(E * N + K)
+    w = oracle.f32_to_bf16(rng.standard_normal((E, N, K)).astype(np.float32) * 0.02)
+    _, s_t, codes, scales = api.qdq_weights(to_bf16_dev(w, cuda), want_qdq=False, want_packed=True)
+    ccm, scm = api.weights_channel_major(codes, scales, N, K)
+    sel = np.sort(rng.choice(K, k, replace=False)).astype(np.int32)
+    seld = torch.from_numpy(sel).to(cuda)
+    a = api.gather_weight_channels(codes, scales, N, K, seld, k, ld)
+    b = api.gather_weight_channels_cm(ccm, scm, N, K, seld, k, ld)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    ccm_n, scm_n = ccm.cpu().numpy(), scm.cpu().numpy()
+    for e in range(E):
+        ref = oracle.quantize(w[e])
+        q = np.empty((N, K), np.uint8)
+        q[:, 0::2] = ref.codes & 0xF
+        q[:, 1::2] = ref.codes >> 4
+        assert np.array_equal(ccm_n[e] & 0xF, q[0::2].T)
+        assert np.array_equal(ccm_n[e] >> 4, q[1::2].T)
+        assert np.array_equal(scm_n[e], ref.sf.T)
+        vals = oracle.e2m1_decode(q) * np.repeat(oracle.e4m3_decode(ref.sf), 16, axis=1)
+        want = oracle.f32_to_bf16(vals[:, sel].astype(np.float32))
+        assert np.array_equal(np_u16(b)[e, :, :k], want)
