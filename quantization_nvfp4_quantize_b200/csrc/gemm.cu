@@ -24,6 +24,11 @@
 // 128, so a tile never spans two experts; the tile count comes from the
 // device-side offsets (no host synchronization).
 //
+// Shared memory: a 4-stage ring of 54 KB stages for the SwiGLU (bf16) epilogue;
+// the f32 epilogues use 3 stages and a 34 KB staging area from which each lane
+// writes 64 contiguous floats of its row with one 256-byte bulk store or bulk
+// add-reduction (cp.reduce.async.bulk .add.f32) -- full-line traffic instead
+// of per-thread 16-byte stores or atomics.
 // TMEM: 512 columns = accumulator [0,256) + scale factors of A [256,272)
 // (4 atoms x 4 columns) + scale factors of B [272,304) (4 x 8 columns).
 // Every mbarrier wait is bounded (1 s); on expiry the kernel records
@@ -41,7 +46,7 @@ namespace gemm {
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int STAGES = 4;
+constexpr int MAX_STAGES = 4;
 constexpr uint32_t A_BYTES = BM * 128;          // 16 KB
 constexpr uint32_t B_BYTES = BN * 128;          // 32 KB
 constexpr uint32_t SFA_BYTES = 4 * 512;         // 4 atoms (K=256 / 64)
@@ -54,7 +59,18 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
 constexpr int MAX_E = 256;
 constexpr uint64_t TIMEOUT_NS = 1000000000ull;
-constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 2048 /*barriers, offsets*/;
+// f32 epilogues stage rows in shared memory and write them with 256-byte bulk
+// copies / bulk add-reductions: per epilogue warp 16 row slots of 64 floats,
+// padded to 68 floats so the 16 writing lanes spread over the banks.
+constexpr uint32_t SLOT_FLOATS = 68;
+constexpr uint32_t STAGING_BYTES = EPI_WARPS * 16 * SLOT_FLOATS * 4;
+
+template <int STAGES>
+struct Cfg {
+    static constexpr bool STAGING = STAGES < MAX_STAGES;      // f32 epilogues give up one stage for staging
+    static constexpr uint32_t SMEM = STAGES * STAGE_BYTES + (STAGING ? STAGING_BYTES : 0) + 1024 /*align*/ +
+                                     2048 /*barriers, offsets*/;
+};
 
 struct Params {
     const uint8_t *a_scales;
@@ -75,8 +91,8 @@ struct Params {
 };
 
 struct Shared {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
     uint64_t tmem_full;
     uint64_t tmem_empty;
     uint64_t drain;
@@ -117,13 +133,16 @@ __device__ __forceinline__ int find_expert(const int *off, int E, int m0)
 
 __device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
+template <int STAGES>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
            const __grid_constant__ CUtensorMap tm_ra, const __grid_constant__ CUtensorMap tm_rb, Params p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *stage_base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Shared *sh = reinterpret_cast<Shared *>(stage_base + STAGES * STAGE_BYTES);
+    float *staging = reinterpret_cast<float *>(stage_base + STAGES * STAGE_BYTES);
+    Shared *sh = reinterpret_cast<Shared *>(stage_base + STAGES * STAGE_BYTES +
+                                            (Cfg<STAGES>::STAGING ? STAGING_BYTES : 0));
     volatile int *abort_flag = &sh->abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -349,6 +368,37 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                     }
                     dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
+            } else if (Cfg<STAGES>::STAGING) {
+                // f32 out: each lane stages 64 contiguous floats of its row and
+                // moves them with one 256-byte bulk store / bulk add-reduction;
+                // lanes 0-15 then 16-31 share the warp's 16 slots.
+                const bool scatter = p.epilogue == MOE_EPI_SCATTER_ADD_F32;
+                const float mul = scatter ? (token >= 0 ? __fmul_rn(scale, p.row_gate[r]) : 0.0f) : scale;
+                float *orow = reinterpret_cast<float *>(p.out) +
+                              (scatter ? (int64_t)(token >= 0 ? token : 0) : r) * p.ld_out + nt * BN + half * 128;
+                float *slot = staging + ((warp - 2) * 16 + (lane & 15)) * SLOT_FLOATS;
+                const uint32_t slot_s = ptx::smem_u32(slot);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        if ((lane >> 4) == rr && token >= 0) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                reinterpret_cast<float4 *>(slot)[j] =
+                                    make_float4(mul * __uint_as_float(v[cc * 64 + 4 * j]),
+                                                mul * __uint_as_float(v[cc * 64 + 4 * j + 1]),
+                                                mul * __uint_as_float(v[cc * 64 + 4 * j + 2]),
+                                                mul * __uint_as_float(v[cc * 64 + 4 * j + 3]));
+                            ptx::fence_proxy_async_smem();
+                            if (scatter) ptx::bulk_reduce_add_f32(orow + cc * 64, slot_s, 256);
+                            else ptx::bulk_store(orow + cc * 64, slot_s, 256);
+                            ptx::bulk_commit();
+                            ptx::bulk_wait_read();          // the slot is reused by the other half-warp
+                        }
+                        __syncwarp();
+                    }
+                }
             } else if (p.epilogue == MOE_EPI_STORE_F32) {
                 if (token >= 0) {
                     float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + r * p.ld_out +
@@ -368,6 +418,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                                                    gw * __uint_as_float(v[4 * j + 2]), gw * __uint_as_float(v[4 * j + 3])));
             }
         }
+        if (Cfg<STAGES>::STAGING) ptx::bulk_wait_all();     // this lane's bulk writes are complete
     }
 
     ptx::tc_fence_before();
@@ -414,7 +465,7 @@ static bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType d
     return r == CUDA_SUCCESS;
 }
 
-static bool smem_attr_done[64];
+static bool smem_attr_done[2][64];
 
 }  // namespace gemm
 }  // namespace nvfp4
@@ -477,12 +528,16 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
     }
     NVFP4_REQUIRE(ok, NVFP4_ERR_CUDA, "moe_w4a4_grouped_gemm_rac: tensor map encoding failed");
 
+    // SwiGLU (bf16 out) keeps 4 stages; the f32 epilogues trade one for staging
+    const bool four = epilogue == MOE_EPI_SWIGLU_BF16;
+    auto kern = four ? k_moe_gemm<4> : k_moe_gemm<3>;
+    const uint32_t smem = four ? Cfg<4>::SMEM : Cfg<3>::SMEM;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !smem_attr_done[dev]) {
-        if (cudaFuncSetAttribute(k_moe_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) != cudaSuccess)
+    if (dev >= 0 && dev < 64 && !smem_attr_done[four][dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return check_launch("moe_w4a4_grouped_gemm_rac: smem attribute");
-        smem_attr_done[dev] = true;
+        smem_attr_done[four][dev] = true;
     }
     Params p{};
     p.a_scales = a_scales_dev;
@@ -504,6 +559,6 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
     int64_t n_tiles = epilogue == MOE_EPI_SWIGLU_BF16 ? inter / 128 : N / BN;
     int64_t max_tiles = (M_pad_max / BM) * n_tiles;
     int grid = (int)std::min<int64_t>(num_sms(), max_tiles);
-    k_moe_gemm<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm_a, tm_b, tm_ra, tm_rb, p);
+    kern<<<grid, NUM_THREADS, smem, st>>>(tm_a, tm_b, tm_ra, tm_rb, p);
     return check_launch("k_moe_gemm");
 }
