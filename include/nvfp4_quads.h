@@ -106,6 +106,11 @@ NVFP4_API int nvfp4_num_sms(void);
  *   m_valid_dev  optional int32 on the device: rows >= *m_valid_dev are
  *                ignored (absent from amax, scores and outputs).  NULL = M.
  *   s_t_in_dev   optional float32: use this tensor scale instead of amax.
+ *   amax_in_dev  optional float32: the tensor's max |x| over its valid rows,
+ *                already computed by the producer of x (e.g. the SwiGLU
+ *                epilogue of moe_w4a4_grouped_gemm_rac); s_t is derived from
+ *                it and the amax pass is skipped.  Ignored when s_t_in_dev is
+ *                given.
  *   s_t_out_dev  float32 [1]: receives s_t (required).
  *   dst_rows_dev optional int32 [M x fanout]: input row r is written to output
  *                rows dst_rows[r*fanout + j] (j < fanout); a negative entry
@@ -129,7 +134,7 @@ NVFP4_API size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K);
 
 NVFP4_API nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
                             const int32_t *m_valid_dev,
-                            const float *s_t_in_dev, float *s_t_out_dev,
+                            const float *s_t_in_dev, const float *amax_in_dev, float *s_t_out_dev,
                             const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
                             uint8_t *codes_dev, uint8_t *scales_dev,
                             double *score_dev, int32_t rac_k, int32_t rac_ld,
@@ -166,7 +171,8 @@ NVFP4_API size_t nvfp4_quantize_noalloc_max_scratch(void);
 
 NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
                                               const int32_t *m_valid_dev,
-                                              const float *s_t_in_dev, float *s_t_out_dev,
+                                              const float *s_t_in_dev, const float *amax_in_dev,
+                                              float *s_t_out_dev,
                                               const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
                                               uint8_t *codes_dev, uint8_t *scales_dev,
                                               double *score_dev, int32_t rac_k, int32_t rac_ld,
@@ -277,7 +283,9 @@ NVFP4_API nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_d
  *                        out bf16 [M_pad_max x ld_out]:
  *                        h[r,i] = bf16(silu(y[r,i]) * y[r,I+i]) for i < I;
  *                        rows with row_token < 0 (and < offsets[E]) are
- *                        written as 0.  I % 128 == 0.
+ *                        written as 0.  I % 128 == 0.  If amax_out_dev is
+ *                        non-NULL it receives max |h| over every row written
+ *                        (the value nvfp4_quantize's amax_in_dev takes).
  *   MOE_EPI_SCATTER_ADD_F32  out f32 [T x ld_out]:
  *                        out[row_token[r], n] += row_gate[r] * y[r,n]
  *                        (atomic; the caller zeroes out first).
@@ -307,7 +315,7 @@ NVFP4_API nvfp4_status moe_w4a4_grouped_gemm_rac(
     const int32_t *offsets_dev,
     int32_t rac_ld, const void *rho_dev, const void *w_sel_dev,
     int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev,
-    void *out_dev, int64_t ld_out,
+    void *out_dev, int64_t ld_out, float *amax_out_dev,
     int32_t *dev_status, void *stream);
 
 /* --------------------------------------------------------------------------

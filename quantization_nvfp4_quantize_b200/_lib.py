@@ -22,12 +22,12 @@ SIGNATURES = {
     "nvfp4_read_status": (c_int32, [c_void_p, c_void_p, c_void_p]),
     "nvfp4_num_sms": (ctypes.c_int, []),
     "nvfp4_quantize_workspace_size": (c_size_t, [c_int64, c_int64]),
-    "nvfp4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+    "nvfp4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_int32, c_int64, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "nvfp4_quantize_noalloc_max_scratch": (c_size_t, []),
     "nvfp4_quantize_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
-                                         c_void_p, c_int32, c_int64, c_void_p, c_void_p, c_void_p, c_int32,
+                                         c_void_p, c_void_p, c_int32, c_int64, c_void_p, c_void_p, c_void_p, c_int32,
                                          c_int32, c_void_p, c_void_p, c_void_p, c_void_p]),
     "nvfp4_qdq_workspace_size": (c_size_t, [c_int64, c_int64, c_int64]),
     "nvfp4_qdq_weights": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
@@ -44,7 +44,7 @@ SIGNATURES = {
     "moe_w4a4_grouped_gemm_rac": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
                                             c_void_p, c_int64, c_int64, c_int32, c_void_p, c_int32, c_void_p,
                                             c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_void_p,
-                                            c_void_p]),
+                                            c_void_p, c_void_p]),
     "nvfp4_debug_encode": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
 }
 

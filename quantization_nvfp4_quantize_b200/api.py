@@ -53,6 +53,7 @@ class Quantized:
 
 
 def quantize(x: torch.Tensor, *, rac_k: int = 0, rac_ld: int | None = None, s_t: torch.Tensor | None = None,
+             amax: torch.Tensor | None = None,
              dst_rows: torch.Tensor | None = None, fanout: int = 1, m_out: int | None = None,
              m_valid: torch.Tensor | None = None, want_score: bool = False, out: Quantized | None = None,
              workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None) -> Quantized:
@@ -76,7 +77,7 @@ def quantize(x: torch.Tensor, *, rac_k: int = 0, rac_ld: int | None = None, s_t:
         )
     if workspace is None:
         workspace = _ws(lib.nvfp4_quantize_workspace_size(M, K), dev)
-    check(lib.nvfp4_quantize(_p(x), M, K, x.stride(0), _p(m_valid), _p(s_t), _p(out.s_t), _p(dst_rows),
+    check(lib.nvfp4_quantize(_p(x), M, K, x.stride(0), _p(m_valid), _p(s_t), _p(amax), _p(out.s_t), _p(dst_rows),
                              fanout, m_out, _p(out.codes), _p(out.scales), _p(out.score), rac_k, rac_ld,
                              _p(out.sel), _p(out.r_sel), _p(dev_status), _p(workspace), workspace.numel(),
                              _stream(dev)))
@@ -170,7 +171,7 @@ def gather_weight_channels_cm(codes_cm: torch.Tensor, scales_cm: torch.Tensor, N
 
 def grouped_gemm(a_codes, a_scales, a_s_t, m_pad_max, b_codes, b_scales, b_s_t, N, K, E, offsets, *,
                  rac_ld=0, rho=None, w_sel=None, epilogue=EPI_STORE_F32, row_token=None, row_gate=None,
-                 out=None, ld_out=None, dev_status=None):
+                 out=None, ld_out=None, amax_out=None, dev_status=None):
     """moe_w4a4_grouped_gemm_rac (see the header)."""
     lib = _lib.load()
     if ld_out is None:
@@ -178,7 +179,7 @@ def grouped_gemm(a_codes, a_scales, a_s_t, m_pad_max, b_codes, b_scales, b_s_t, 
     check(lib.moe_w4a4_grouped_gemm_rac(_p(a_codes), _p(a_scales), _p(a_s_t), m_pad_max, _p(b_codes),
                                         _p(b_scales), _p(b_s_t), N, K, E, _p(offsets), rac_ld, _p(rho),
                                         _p(w_sel), epilogue, _p(row_token), _p(row_gate), _p(out), ld_out,
-                                        _p(dev_status), _stream(out.device)))
+                                        _p(amax_out), _p(dev_status), _stream(out.device)))
     return out
 
 

@@ -10,6 +10,7 @@
 // Host side: error strings, argument checks, launch checks.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -26,6 +27,11 @@ namespace nvfp4 {
 nvfp4_status set_error(nvfp4_status st, const char *fmt, ...);
 nvfp4_status check_launch(const char *what);
 int num_sms();
+
+// Row-major 2D tensor [rows x inner] (row stride row_bytes) with a
+// (box_inner x box_rows) TMA box; false if the driver rejects it.
+bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t inner, uint64_t rows,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle);
 
 #define NVFP4_REQUIRE(cond, status, ...)                 \
     do {                                                 \

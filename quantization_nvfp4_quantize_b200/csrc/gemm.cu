@@ -87,6 +87,7 @@ struct Params {
     const float *row_gate;
     void *out;
     int64_t ld_out;
+    unsigned int *amax_out;    // SwiGLU: max |h| (float bits), or null
     int32_t *dev_status;
 };
 
@@ -352,6 +353,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             if (p.epilogue == MOE_EPI_SWIGLU_BF16) {
                 uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + r * p.ld_out +
                                                        nt * 128 + half * 64);
+                float hmax = 0.0f;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint32_t w4[4];
@@ -363,10 +365,16 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                             h0 = silu(scale * __uint_as_float(v[j])) * (scale * __uint_as_float(v[64 + j]));
                             h1 = silu(scale * __uint_as_float(v[j + 1])) * (scale * __uint_as_float(v[64 + j + 1]));
                         }
-                        w4[jj] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h0)) |
-                                 ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h1)) << 16);
+                        const __nv_bfloat16 b0 = __float2bfloat16_rn(h0), b1 = __float2bfloat16_rn(h1);
+                        hmax = fmaxf(hmax, fmaxf(fabsf(__bfloat162float(b0)), fabsf(__bfloat162float(b1))));
+                        w4[jj] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
                     }
                     dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+                if (p.amax_out) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+                    if (lane == 0) atomicMax(p.amax_out, __float_as_uint(hmax));
                 }
             } else if (Cfg<STAGES>::STAGING) {
                 // f32 out: each lane stages 64 contiguous floats of its row and
@@ -431,40 +439,6 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
 
 // ----------------------------------------------------------------- host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    });
-    return fn;
-}
-
-// Row-major 2D tensor [rows x inner] with a (box_inner x box_rows) box and
-// 128-byte swizzle.
-static bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t inner, uint64_t rows,
-                         uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 static bool smem_attr_done[2][64];
 
 }  // namespace gemm
@@ -476,8 +450,8 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
     const uint8_t *a_codes_dev, const uint8_t *a_scales_dev, const float *a_s_t_dev, int64_t M_pad_max,
     const uint8_t *b_codes_dev, const uint8_t *b_scales_dev, const float *b_s_t_dev, int64_t N, int64_t K, int32_t E,
     const int32_t *offsets_dev, int32_t rac_ld, const void *rho_dev, const void *w_sel_dev, int32_t epilogue,
-    const int32_t *row_token_dev, const float *row_gate_dev, void *out_dev, int64_t ld_out, int32_t *dev_status,
-    void *stream)
+    const int32_t *row_token_dev, const float *row_gate_dev, void *out_dev, int64_t ld_out, float *amax_out_dev,
+    int32_t *dev_status, void *stream)
 {
     using namespace nvfp4::gemm;
     cudaStream_t st = (cudaStream_t)stream;
@@ -513,15 +487,16 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
                   NVFP4_ERR_ALIGNMENT, "moe_w4a4_grouped_gemm_rac: pointers must be 16-byte aligned");
 
     CUtensorMap tm_a, tm_b, tm_ra, tm_rb;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     bool ok = make_tmap_2d(&tm_a, a_codes_dev, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)M_pad_max,
-                           (uint64_t)K / 2, 128, 128) &&
+                           (uint64_t)K / 2, 128, 128, sw) &&
               make_tmap_2d(&tm_b, b_codes_dev, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)E * N,
-                           (uint64_t)K / 2, 128, 128);
+                           (uint64_t)K / 2, 128, 128, sw);
     if (ok && rac_ld > 0) {
         ok = make_tmap_2d(&tm_ra, rho_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)rac_ld, (uint64_t)M_pad_max,
-                          (uint64_t)rac_ld * 2, 64, 128) &&
+                          (uint64_t)rac_ld * 2, 64, 128, sw) &&
              make_tmap_2d(&tm_rb, w_sel_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)rac_ld, (uint64_t)E * N,
-                          (uint64_t)rac_ld * 2, 64, 128);
+                          (uint64_t)rac_ld * 2, 64, 128, sw);
     } else {
         tm_ra = tm_a;
         tm_rb = tm_b;
@@ -555,7 +530,10 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
     p.row_gate = row_gate_dev;
     p.out = out_dev;
     p.ld_out = ld_out;
+    p.amax_out = (epilogue == MOE_EPI_SWIGLU_BF16) ? reinterpret_cast<unsigned int *>(amax_out_dev) : nullptr;
     p.dev_status = dev_status;
+    if (p.amax_out && cudaMemsetAsync(p.amax_out, 0, sizeof(float), st) != cudaSuccess)
+        return check_launch("moe_w4a4_grouped_gemm_rac: memset");
     int64_t n_tiles = epilogue == MOE_EPI_SWIGLU_BF16 ? inter / 128 : N / BN;
     int64_t max_tiles = (M_pad_max / BM) * n_tiles;
     int grid = (int)std::min<int64_t>(num_sms(), max_tiles);

@@ -20,6 +20,7 @@
 // 8 warps in shared memory and writes one partial per channel; partials are
 // summed in a fixed order by k_score_reduce, so scores are deterministic.
 #include "common.cuh"
+#include "ptx.cuh"
 
 #include <algorithm>
 #include <mutex>
@@ -28,9 +29,10 @@ namespace nvfp4 {
 
 constexpr int QTHREADS = 256;
 constexpr int QCHUNK = 256;           // channels per CTA column chunk
-constexpr int QCTAS_PER_SM = 4;       // resident CTAs per SM the grid is sized for (one wave)
-constexpr int ROWS_IN_FLIGHT = 4;     // rows a warp loads before processing them; also the
-                                      // number of rows summed in binary32 before binary64
+constexpr int QCTAS_PER_SM = 3;       // resident CTAs per SM the grid is sized for (one wave)
+constexpr int QSTAGES = 4;            // TMA tile ring depth
+constexpr int QROWS = 32;             // rows per TMA tile
+constexpr uint32_t QSMEM = QSTAGES * QROWS * QCHUNK * 2;   // 64 KB of tiles per CTA
 
 // -------------------------------------------------------------------- amax
 
@@ -73,11 +75,10 @@ __global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16 *__restrict__ 
 // --------------------------------------------------------------- quantize
 
 struct QuantParams {
-    const __nv_bfloat16 *x;
     int64_t ldx, M, K;
     const int32_t *m_valid;
     const float *s_t_in;             // per group, or null
-    const unsigned int *amax_bits;   // per group, used when s_t_in is null
+    const unsigned int *amax_bits;   // per group (max |x| as float bits), used when s_t_in is null
     float *s_t_out;                  // per group
     const int32_t *dst_rows;
     int fanout;
@@ -86,17 +87,53 @@ struct QuantParams {
     __nv_bfloat16 *qdq;
     double *partials;                // [gridDim.y x K]
     int64_t rows_per_cta;
-    int64_t x_gstride, codes_gstride, scales_gstride, qdq_gstride;
+    int64_t codes_gstride, scales_gstride, qdq_gstride;
+    int box_inner;                   // channels per TMA box row (min(256, K))
+    int32_t *dev_status;
 };
 
-template <bool SCORE>
-__global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(QuantParams p)
+// Bounded mbarrier wait for the streaming kernels (1 s); false on timeout or
+// when another thread of the CTA has given up.
+__device__ __forceinline__ bool qwait(uint32_t bar, uint32_t parity, volatile int *abort_flag, int32_t *dev_status,
+                                      bool ignore_abort = false)
 {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 63u) {
+            if (!ignore_abort && *abort_flag) return false;
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > 1000000000ull) {
+                *abort_flag = 1;
+                report_status(dev_status, NVFP4_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// One CTA = 8 warps on one 256-channel column chunk and one range of rows.
+// Thread 0 streams 32-row x 256-channel bf16 tiles (16 KB) through a 4-stage
+// shared-memory ring with TMA; warp w quantizes tile rows w, w+8, w+16, w+24,
+// each lane 8 channels (a lane pair is one 16-element block).
+template <bool SCORE>
+__global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __grid_constant__ CUtensorMap tm_x,
+                                                                     QuantParams p)
+{
+    extern __shared__ __align__(128) uint8_t qsm[];              // QSTAGES x QROWS x box_inner bf16
+    __shared__ uint64_t full_bar[QSTAGES], empty_bar[QSTAGES];
+    __shared__ int abort_sm;
+    volatile int *abort_flag = &abort_sm;
+
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = blockIdx.z;
     const int64_t K = p.K;
-    const int64_t c = (int64_t)blockIdx.x * QCHUNK + lane * 8;   // first channel of this lane
+    const int64_t c0 = (int64_t)blockIdx.x * QCHUNK;
+    const int64_t c = c0 + lane * 8;                              // first channel of this lane
     const bool active = c < K;
+    const uint32_t pitch = (uint32_t)p.box_inner * 2u;            // bytes per tile row in shared memory
+    const uint32_t tile_bytes = pitch * QROWS;
 
     float s_t = p.s_t_in ? p.s_t_in[g] : tensor_scale_from_amax(__uint_as_float(p.amax_bits[g]));
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.s_t_out) p.s_t_out[g] = s_t;
@@ -106,11 +143,33 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(QuantParams
     if (p.m_valid) Me = min(Me, (int64_t)max(*p.m_valid, 0));
     const int64_t r0 = (int64_t)blockIdx.y * p.rows_per_cta;
     const int64_t r1 = min(Me, r0 + p.rows_per_cta);
+    const int n_iter = r1 > r0 ? (int)((r1 - r0 + QROWS - 1) / QROWS) : 0;
+    const int64_t row_base = (int64_t)g * p.M;                   // row of this group in the tensor map
 
-    const __nv_bfloat16 *xg = p.x + g * p.x_gstride;
     uint8_t *codes = p.codes ? p.codes + g * p.codes_gstride : nullptr;
     uint8_t *scales = p.scales ? p.scales + g * p.scales_gstride : nullptr;
     __nv_bfloat16 *qdq = p.qdq ? p.qdq + g * p.qdq_gstride : nullptr;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < QSTAGES; ++st) {
+            ptx::mbar_init(ptx::smem_u32(&full_bar[st]), 1);
+            ptx::mbar_init(ptx::smem_u32(&empty_bar[st]), QTHREADS / 32);
+        }
+        abort_sm = 0;
+        ptx::fence_mbar_init();
+        ptx::fence_proxy_async_smem();
+    }
+    __syncthreads();
+    int issued = 0;                                               // thread 0 only
+    if (threadIdx.x == 0) {
+        ptx::prefetch_tmap(&tm_x);
+        for (; issued < min(n_iter, QSTAGES); ++issued) {
+            const uint32_t fb = ptx::smem_u32(&full_bar[issued]);
+            ptx::mbar_arrive_expect_tx(fb, tile_bytes);
+            ptx::tma_load_2d(ptx::smem_u32(qsm + issued * tile_bytes), &tm_x, (int32_t)c0,
+                             (int32_t)(row_base + r0 + (int64_t)issued * QROWS), fb);
+        }
+    }
 
     float acc32[8];
     double acc64[8];
@@ -118,23 +177,24 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(QuantParams
     for (int i = 0; i < 8; ++i) { acc32[i] = 0.0f; acc64[i] = 0.0; }
 
     const int64_t kb0 = c >> 4;                 // first block of the 4-block group (lanes 8j)
-    constexpr int WARPS = QTHREADS / 32;
-    for (int64_t rbase = r0 + warp; rbase < r1; rbase += ROWS_IN_FLIGHT * WARPS) {
-        // issue every row's load first: ROWS_IN_FLIGHT 16-byte loads per lane in flight
-        uint4 u[ROWS_IN_FLIGHT];
+    int it = 0;
+    for (; it < n_iter; ++it) {
+        const int st = it % QSTAGES;
+        const uint32_t ph = (uint32_t)(it / QSTAGES) & 1u;
+        bool ok = true;
+        if (lane == 0) ok = qwait(ptx::smem_u32(&full_bar[st]), ph, abort_flag, p.dev_status);
+        if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
+        const uint8_t *tile = qsm + st * tile_bytes;
 #pragma unroll
-        for (int i = 0; i < ROWS_IN_FLIGHT; ++i) {
-            const int64_t r = rbase + (int64_t)i * WARPS;
-            u[i] = (active && r < r1) ? __ldg(reinterpret_cast<const uint4 *>(xg + r * p.ldx + c))
-                                      : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int i = 0; i < ROWS_IN_FLIGHT; ++i) {
-            const int64_t r = rbase + (int64_t)i * WARPS;
-            if (r >= r1) break;                 // warp-uniform
+        for (int i = 0; i < QROWS / (QTHREADS / 32); ++i) {
+            const int lr = warp + i * (QTHREADS / 32);            // row inside the tile
+            const int64_t r = r0 + (int64_t)it * QROWS + lr;
+            if (r >= r1) break;                                   // warp-uniform
+            uint4 u = active ? *reinterpret_cast<const uint4 *>(tile + lr * pitch + lane * 16)
+                             : make_uint4(0u, 0u, 0u, 0u);
             float v[8];
-            v[0] = bf16lo(u[i].x); v[1] = bf16hi(u[i].x); v[2] = bf16lo(u[i].y); v[3] = bf16hi(u[i].y);
-            v[4] = bf16lo(u[i].z); v[5] = bf16hi(u[i].z); v[6] = bf16lo(u[i].w); v[7] = bf16hi(u[i].w);
+            v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+            v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
             float m = fabsf(v[0]);
 #pragma unroll
             for (int k = 1; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
@@ -182,23 +242,41 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(QuantParams
             }
         }
         if (SCORE) {
-            // at most ROWS_IN_FLIGHT rows were summed in binary32
+            // at most QROWS / 8 = 4 rows were summed in binary32
 #pragma unroll
             for (int k = 0; k < 8; ++k) { acc64[k] += (double)acc32[k]; acc32[k] = 0.0f; }
         }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty_bar[st]));
+        if (threadIdx.x == 0 && issued < n_iter) {
+            // refill this slot once every warp has consumed it
+            if (!qwait(ptx::smem_u32(&empty_bar[st]), ph, abort_flag, p.dev_status)) break;
+            const uint32_t fb = ptx::smem_u32(&full_bar[st]);
+            ptx::mbar_arrive_expect_tx(fb, tile_bytes);
+            ptx::tma_load_2d(ptx::smem_u32(qsm + st * tile_bytes), &tm_x, (int32_t)c0,
+                             (int32_t)(row_base + r0 + (int64_t)issued * QROWS), fb);
+            ++issued;
+        }
+    }
+    if (threadIdx.x == 0) {
+        // after an early exit, let every issued copy land before the CTA ends
+        for (int j = it; j < issued; ++j)
+            qwait(ptx::smem_u32(&full_bar[j % QSTAGES]), (uint32_t)(j / QSTAGES) & 1u, abort_flag, p.dev_status,
+                  true);
     }
 
     if (SCORE) {
-        __shared__ double red[QTHREADS / 32][QCHUNK];
+        __syncthreads();                                          // the stage ring is free: reuse it
+        double *red = reinterpret_cast<double *>(qsm);            // [8 warps][256 channels]
 #pragma unroll
-        for (int i = 0; i < 8; ++i) red[warp][lane * 8 + i] = acc64[i] + (double)acc32[i];
+        for (int i = 0; i < 8; ++i) red[warp * QCHUNK + lane * 8 + i] = acc64[i] + (double)acc32[i];
         __syncthreads();
-        int64_t ch = (int64_t)blockIdx.x * QCHUNK + threadIdx.x;
+        int64_t ch = c0 + threadIdx.x;
         if (ch < K) {
-            double s = 0.0;
+            double sum = 0.0;
 #pragma unroll
-            for (int w = 0; w < QTHREADS / 32; ++w) s += red[w][threadIdx.x];
-            p.partials[(int64_t)blockIdx.y * K + ch] = s;
+            for (int w = 0; w < QTHREADS / 32; ++w) sum += red[w * QCHUNK + threadIdx.x];
+            p.partials[(int64_t)blockIdx.y * K + ch] = sum;
         }
     }
 }
@@ -441,7 +519,7 @@ __global__ void k_weights_channel_major(const uint8_t *__restrict__ codes, const
 // bf16) into a shared [channel][feature] tile, then written out transposed as
 // [feature][ld] rows.
 constexpr int GCM_N = 64;
-constexpr int GCM_TS = GCM_N + 1;                     // padded row of the shared tile (floats)
+constexpr int GCM_TS = GCM_N + 4;                     // padded row of the shared tile (floats)
 
 __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__restrict__ codes_cm,
                                                               const uint8_t *__restrict__ scales_cm, int64_t N,
@@ -451,28 +529,39 @@ __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__r
     extern __shared__ float gtile[];                   // [ld][GCM_TS]
     const int64_t e = blockIdx.y;
     const int64_t n0 = (int64_t)blockIdx.x * GCM_N;
-    // phase 1: thread (j, f) dequantizes feature n0 + f of selected channel j
-    for (int idx = threadIdx.x; idx < ld * GCM_N; idx += blockDim.x) {
-        const int jj = idx / GCM_N;
-        const int f = idx - jj * GCM_N;
-        float v = 0.0f;
+    // phase 1: thread (j, 8 features): one 4-byte code load, one 8-byte scale load
+    for (int idx = threadIdx.x; idx < ld * (GCM_N / 8); idx += blockDim.x) {
+        const int jj = idx / (GCM_N / 8);
+        const int f0 = (idx - jj * (GCM_N / 8)) * 8;
+        float v[8];
         if (jj < k) {
             const int64_t ch = sel[jj];
-            const int64_t n = n0 + f;
-            const uint32_t byte = codes_cm[(e * K + ch) * (N / 2) + (n >> 1)];
-            const uint32_t nib = (n & 1) ? (byte >> 4) : (byte & 15u);
-            const float q = e2m1x2_to_f32(nib).x;
-            const float sf = e4m3_to_f32(scales_cm[(e * (K / 16) + (ch >> 4)) * N + n]);
-            v = __fmul_rn(q, sf);
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(codes_cm + (e * K + ch) * (N / 2) + (n0 + f0) / 2);
+            const uint2 sc = *reinterpret_cast<const uint2 *>(scales_cm + (e * (K / 16) + (ch >> 4)) * N + n0 + f0);
+            float q[8];
+            e2m1x8_to_f32(w, q);
+            const uint32_t sw[2] = {sc.x, sc.y};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(q[i], e4m3_to_f32((sw[i >> 2] >> (8 * (i & 3))) & 0xFFu));
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
         }
-        gtile[jj * GCM_TS + f] = v;
+        float4 *dst = reinterpret_cast<float4 *>(gtile + jj * GCM_TS + f0);
+        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
     }
     __syncthreads();
-    // phase 2: thread (f, j) writes out[e, n0 + f, j]; consecutive threads take consecutive j
-    for (int idx = threadIdx.x; idx < GCM_N * ld; idx += blockDim.x) {
-        const int f = idx / ld;
-        const int jj = idx - f * ld;
-        out[(e * N + n0 + f) * ld + jj] = __float2bfloat16_rn(gtile[jj * GCM_TS + f]);
+    // phase 2: thread (feature f, 8 channels) writes 16 bytes of out[e, n0 + f, :]
+    for (int idx = threadIdx.x; idx < GCM_N * (ld / 8); idx += blockDim.x) {
+        const int f = idx / (ld / 8);
+        const int j0 = (idx - f * (ld / 8)) * 8;
+        uint32_t pk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            pk[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(gtile[(j0 + 2 * i) * GCM_TS + f])) |
+                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(gtile[(j0 + 2 * i + 1) * GCM_TS + f])) << 16);
+        *reinterpret_cast<uint4 *>(out + (e * N + n0 + f) * ld + j0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
 }
 
@@ -489,6 +578,36 @@ static int64_t pick_rows_per_cta(int64_t M, int64_t nchunks, int64_t groups)
 }
 
 static int64_t row_groups(int64_t M, int64_t rpc) { return std::max<int64_t>(1, (M + rpc - 1) / rpc); }
+
+// Builds the TMA map over x ([rows_total x K] bf16, row stride ldx) and
+// launches k_quantize.  `fallback` is any valid 16-byte aligned device
+// address, used as the map's base when x has no rows (no copy is issued then).
+static nvfp4_status launch_quantize(bool score, const void *x, int64_t rows_total, const void *fallback,
+                                    QuantParams &p, dim3 grid, cudaStream_t st)
+{
+    static bool attr_done[2][64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[score][dev]) {
+        cudaError_t e = score ? cudaFuncSetAttribute(k_quantize<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)QSMEM)
+                              : cudaFuncSetAttribute(k_quantize<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)QSMEM);
+        if (e != cudaSuccess) return check_launch("k_quantize: smem attribute");
+        attr_done[score][dev] = true;
+    }
+    p.box_inner = (int)std::min<int64_t>(QCHUNK, p.K);
+    CUtensorMap tm;
+    const bool empty = rows_total <= 0 || x == nullptr;
+    if (!make_tmap_2d(&tm, empty ? fallback : x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)p.K,
+                      (uint64_t)(empty ? 1 : rows_total), (uint64_t)p.ldx * 2, (uint32_t)p.box_inner, QROWS,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+        return set_error(NVFP4_ERR_CUDA, "k_quantize: tensor map encoding failed");
+    const size_t smem = (size_t)QSTAGES * QROWS * p.box_inner * 2;
+    if (score) k_quantize<true><<<grid, QTHREADS, smem, st>>>(tm, p);
+    else k_quantize<false><<<grid, QTHREADS, smem, st>>>(tm, p);
+    return check_launch("k_quantize");
+}
 
 }  // namespace nvfp4
 
@@ -507,7 +626,7 @@ extern "C" size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K)
 
 extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
                                        const int32_t *m_valid_dev,
-                                       const float *s_t_in_dev, float *s_t_out_dev,
+                                       const float *s_t_in_dev, const float *amax_in_dev, float *s_t_out_dev,
                                        const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
                                        uint8_t *codes_dev, uint8_t *scales_dev,
                                        double *score_dev, int32_t rac_k, int32_t rac_ld,
@@ -515,7 +634,6 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
                                        int32_t *dev_status, void *workspace, size_t workspace_bytes,
                                        void *stream)
 {
-    (void)dev_status;
     cudaStream_t st = (cudaStream_t)stream;
     NVFP4_REQUIRE(M >= 0 && K > 0 && M_out >= 0, NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: bad sizes");
     NVFP4_REQUIRE(s_t_out_dev && (M == 0 || x_dev) && (M_out == 0 || (codes_dev && scales_dev)),
@@ -544,23 +662,26 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
     NVFP4_REQUIRE(workspace && workspace_bytes >= need && aligned16(workspace), NVFP4_ERR_WORKSPACE,
                   "nvfp4_quantize: workspace of %zu bytes (16-byte aligned) required", need);
 
-    unsigned int *amax_bits = reinterpret_cast<unsigned int *>(workspace);
+    // non-negative floats order like their bit patterns: a precomputed max |x|
+    // is read through the same unsigned view as the amax pass's result
+    const unsigned int *amax_bits = amax_in_dev ? reinterpret_cast<const unsigned int *>(amax_in_dev)
+                                                : reinterpret_cast<unsigned int *>(workspace);
     const int64_t nch = (K + QCHUNK - 1) / QCHUNK;
     const int64_t rpc = pick_rows_per_cta(M, nch, 1);
     const int64_t P = row_groups(M, rpc);
     double *partials = reinterpret_cast<double *>(reinterpret_cast<char *>(workspace) + 256);
     double *score = score_dev ? score_dev : partials + P * K;
 
-    if (!s_t_in_dev) {
-        if (cudaMemsetAsync(amax_bits, 0, 4, st) != cudaSuccess) return check_launch("nvfp4_quantize: memset");
+    if (!s_t_in_dev && !amax_in_dev) {
+        unsigned int *slot = reinterpret_cast<unsigned int *>(workspace);
+        if (cudaMemsetAsync(slot, 0, 4, st) != cudaSuccess) return check_launch("nvfp4_quantize: memset");
         if (M > 0) {
             int blocks = (int)std::min<int64_t>((int64_t)num_sms() * 8, std::max<int64_t>(1, (M * K / 8 + 255) / 256));
-            k_amax<<<dim3(blocks, 1), 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, 0, amax_bits);
+            k_amax<<<dim3(blocks, 1), 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, 0, slot);
             if (check_launch("k_amax") != NVFP4_OK) return NVFP4_ERR_CUDA;
         }
     }
     QuantParams p{};
-    p.x = (const __nv_bfloat16 *)x_dev;
     p.ldx = ldx; p.M = M; p.K = K;
     p.m_valid = m_valid_dev;
     p.s_t_in = s_t_in_dev;
@@ -573,10 +694,9 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
     p.qdq = nullptr;
     p.partials = partials;
     p.rows_per_cta = rpc;
+    p.dev_status = dev_status;
     dim3 grid((unsigned)nch, (unsigned)P, 1);
-    if (want_score) k_quantize<true><<<grid, QTHREADS, 0, st>>>(p);
-    else k_quantize<false><<<grid, QTHREADS, 0, st>>>(p);
-    if (check_launch("k_quantize") != NVFP4_OK) return NVFP4_ERR_CUDA;
+    if (launch_quantize(want_score, x_dev, M, workspace, p, grid, st) != NVFP4_OK) return NVFP4_ERR_CUDA;
 
     if (want_score) {
         k_score_reduce<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(partials, P, K, score);
@@ -646,7 +766,6 @@ extern "C" nvfp4_status nvfp4_qdq_weights(const void *w_dev, int64_t G, int64_t 
     const int64_t nch = (cols + QCHUNK - 1) / QCHUNK;
     const int64_t rpc = pick_rows_per_cta(rows, nch, G);
     QuantParams p{};
-    p.x = (const __nv_bfloat16 *)w_dev;
     p.ldx = cols; p.M = rows; p.K = cols;
     p.amax_bits = amax_bits;
     p.s_t_out = s_t_dev;
@@ -655,13 +774,11 @@ extern "C" nvfp4_status nvfp4_qdq_weights(const void *w_dev, int64_t G, int64_t 
     p.scales = scales_dev;
     p.qdq = (__nv_bfloat16 *)w_qdq_dev;
     p.rows_per_cta = rpc;
-    p.x_gstride = per_group;
     p.codes_gstride = per_group / 2;
     p.scales_gstride = sf_bytes(rows, cols);
     p.qdq_gstride = per_group;
     dim3 grid((unsigned)nch, (unsigned)row_groups(rows, rpc), (unsigned)G);
-    k_quantize<false><<<grid, QTHREADS, 0, st>>>(p);
-    return check_launch("k_quantize (qdq)");
+    return launch_quantize(false, w_dev, G * rows, workspace, p, grid, st);
 }
 
 extern "C" nvfp4_status nvfp4_gather_weight_channels(const uint8_t *codes_dev, const uint8_t *scales_dev,
@@ -798,7 +915,8 @@ extern "C" size_t nvfp4_quantize_noalloc_max_scratch(void) { return nvfp4::NOALL
 
 extern "C" nvfp4_status nvfp4_quantize_noalloc(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
                                                const int32_t *m_valid_dev,
-                                               const float *s_t_in_dev, float *s_t_out_dev,
+                                               const float *s_t_in_dev, const float *amax_in_dev,
+                                               float *s_t_out_dev,
                                                const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
                                                uint8_t *codes_dev, uint8_t *scales_dev,
                                                double *score_dev, int32_t rac_k, int32_t rac_ld,
@@ -814,7 +932,8 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void *x_dev, int64_t M, int
     nvfp4_status st;
     void *scratch = nvfp4::noalloc_scratch_ptr(&st);
     if (!scratch) return st;
-    return nvfp4_quantize(x_dev, M, K, ldx, m_valid_dev, s_t_in_dev, s_t_out_dev, dst_rows_dev, fanout, M_out,
+    return nvfp4_quantize(x_dev, M, K, ldx, m_valid_dev, s_t_in_dev, amax_in_dev, s_t_out_dev, dst_rows_dev, fanout,
+                          M_out,
                           codes_dev, scales_dev, score_dev, rac_k, rac_ld, sel_dev, r_sel_dev, dev_status, scratch,
                           nvfp4::NOALLOC_SCRATCH_BYTES, stream);
 }

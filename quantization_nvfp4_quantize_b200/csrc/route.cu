@@ -32,37 +32,49 @@ __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ lo
         l[i] = (e < E) ? logits[t * E + e] : -INFINITY;
     }
     unsigned taken = 0;      // bit i: expert lane + 32 i already selected
-    float sel_l[MAX_TOPK];
+    float sel_l[MAX_TOPK];   // fully unrolled below: stays in registers
     int sel_e[MAX_TOPK];
-    for (int j = 0; j < kr; ++j) {
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-            int e = lane + 32 * i;
-            if (e < E && !((taken >> i) & 1u)) {
-                if (be == 0x7fffffff || l[i] > bv) { bv = l[i]; be = e; }
+    for (int j = 0; j < MAX_TOPK; ++j) {
+        sel_l[j] = -INFINITY;
+        sel_e[j] = 0;
+        if (j < kr) {
+            float bv = -INFINITY;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+                int e = lane + 32 * i;
+                if (e < E && !((taken >> i) & 1u)) {
+                    if (be == 0x7fffffff || l[i] > bv) { bv = l[i]; be = e; }
+                }
             }
-        }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
+            for (int o = 16; o > 0; o >>= 1) {
+                float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
+            }
+            sel_l[j] = bv;
+            sel_e[j] = be;
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
         }
-        sel_l[j] = bv;
-        sel_e[j] = be;
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
     }
     if (lane == 0) {
-        float mx = sel_l[0];
+        const float mx = sel_l[0];
         float z = 0.0f;
         float ex[MAX_TOPK];
-        for (int j = 0; j < kr; ++j) { ex[j] = expf(sel_l[j] - mx); z += ex[j]; }
-        for (int j = 0; j < kr; ++j) {
-            topk_idx[t * kr + j] = sel_e[j];
-            topk_gate[t * kr + j] = ex[j] / z;
-            atomicAdd(counts + sel_e[j], 1);
+#pragma unroll
+        for (int j = 0; j < MAX_TOPK; ++j) {
+            ex[j] = j < kr ? expf(sel_l[j] - mx) : 0.0f;
+            z += ex[j];
+        }
+#pragma unroll
+        for (int j = 0; j < MAX_TOPK; ++j) {
+            if (j < kr) {
+                topk_idx[t * kr + j] = sel_e[j];
+                topk_gate[t * kr + j] = ex[j] / z;
+                atomicAdd(counts + sel_e[j], 1);
+            }
         }
     }
 }

@@ -9,8 +9,9 @@ and 2.2 B; shd-paper.top abstract):
                                RAC residual rho_x for every routed row
   3. gather_weight_channels_cm W13q[:, :, S_x] as bf16 (e2m1 * sf), read from
                                the channel-major weight copy
-  4. grouped GEMM (gate/up)    W4A4 + RAC, epilogue SwiGLU -> h bf16
-  5. nvfp4_quantize(h)         over the valid routed rows: s_h, codes, S_h, rho_h
+  4. grouped GEMM (gate/up)    W4A4 + RAC, epilogue SwiGLU -> h bf16 and max |h|
+  5. nvfp4_quantize(h)         over the valid routed rows, s_h from the epilogue's
+                               max |h| (no amax pass): codes, S_h, rho_h
   6. gather_weight_channels_cm W2q[:, :, S_h]
   7. grouped GEMM (down)       W4A4 + RAC, epilogue router-weighted scatter-add
                                into Y [T x H] fp32
@@ -61,6 +62,7 @@ class MoELayerW4A4:
         self.w_sel2 = torch.empty(E, H, ld, dtype=torch.bfloat16, device=dev)
         self.h = torch.empty(mp, I, dtype=torch.bfloat16, device=dev)
         self.y = torch.empty(tokens, H, dtype=torch.float32, device=dev)
+        self.h_amax = torch.empty(1, dtype=torch.float32, device=dev)
         lib = api._lib.load()
         self.ws_x = api._ws(lib.nvfp4_quantize_workspace_size(tokens, H), dev)
         self.ws_h = api._ws(lib.nvfp4_quantize_workspace_size(mp, I), dev)
@@ -78,9 +80,9 @@ class MoELayerW4A4:
         api.grouped_gemm(self.xq.codes, self.xq.scales, self.xq.s_t, self.m_pad, self.c13, self.sf13, self.s13,
                          2 * I, H, E, r.offsets, rac_ld=self.rac_ld if k else 0, rho=self.xq.r_sel,
                          w_sel=self.w_sel13, epilogue=api.EPI_SWIGLU_BF16, row_token=r.row_token,
-                         row_gate=r.row_gate, out=self.h)
+                         row_gate=r.row_gate, out=self.h, amax_out=self.h_amax)
         api.quantize(self.h, rac_k=k, rac_ld=self.rac_ld, m_out=self.m_pad, m_valid=r.offsets[E:],
-                     out=self.hq, workspace=self.ws_h)
+                     amax=self.h_amax, out=self.hq, workspace=self.ws_h)
         if k:
             api.gather_weight_channels_cm(self.c2_cm, self.sf2_cm, H, I, self.hq.sel, k, self.rac_ld,
                                           out=self.w_sel2)

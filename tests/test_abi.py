@@ -49,25 +49,25 @@ def _status(fn, *args):
 def test_argument_errors_are_synchronous():
     lib = _lib.load()
     # null input
-    st = lib.nvfp4_quantize(None, 4, 64, 64, None, None, None, None, 1, 4, None, None, None, 0, 0, None, None,
+    st = lib.nvfp4_quantize(None, 4, 64, 64, None, None, None, None, None, 1, 4, None, None, None, 0, 0, None, None,
                             None, None, 0, None)
     assert st == 1 and b"required" in lib.nvfp4_last_error_string()
     fake = ctypes.c_void_p(0x10000)          # never dereferenced: rejected before any launch
     # K not a multiple of 64
-    st = lib.nvfp4_quantize(fake, 4, 48, 48, None, None, fake, None, 1, 4, fake, fake, None, 0, 0, None, None,
+    st = lib.nvfp4_quantize(fake, 4, 48, 48, None, None, None, fake, None, 1, 4, fake, fake, None, 0, 0, None, None,
                             None, fake, 1 << 20, None)
     assert st == 3
     # misaligned pointer
-    st = lib.nvfp4_quantize(ctypes.c_void_p(0x10008), 4, 64, 64, None, None, fake, None, 1, 4, fake, fake, None,
+    st = lib.nvfp4_quantize(ctypes.c_void_p(0x10008), 4, 64, 64, None, None, None, fake, None, 1, 4, fake, fake, None,
                             0, 0, None, None, None, fake, 1 << 20, None)
     assert st == 2
     # rac_k too large
-    st = lib.nvfp4_quantize(fake, 4, 64, 64, None, None, fake, None, 1, 4, fake, fake, fake, 65, 128, fake, fake,
+    st = lib.nvfp4_quantize(fake, 4, 64, 64, None, None, None, fake, None, 1, 4, fake, fake, fake, 65, 128, fake, fake,
                             None, fake, 1 << 20, None)
     assert st == 3
     # GEMM shape errors
     args = [fake, fake, fake, 128, fake, fake, fake, 256, 256, 1, fake, 0, None, None, 0, fake, fake, fake, 256,
-            None, None]
+            None, None, None]
     bad_k = list(args)
     bad_k[8] = 320
     assert lib.moe_w4a4_grouped_gemm_rac(*bad_k) == 3

@@ -95,9 +95,10 @@ def test_gemm_swiglu_and_scatter(cuda):
     N = 2 * I
     x, w, logits, r, xq, s_w, c_w, sf_w, w_sel, rac_ld = _setup(cuda, rng, T, E, kr, N, K, rac_k)
     h = torch.full((r.m_pad_max, I), float("nan"), dtype=torch.bfloat16, device=cuda)
+    h_amax = torch.full((1,), 123.0, dtype=torch.float32, device=cuda)
     api.grouped_gemm(xq.codes, xq.scales, xq.s_t, r.m_pad_max, c_w, sf_w, s_w, N, K, E, r.offsets,
                      rac_ld=rac_ld, rho=xq.r_sel, w_sel=w_sel, epilogue=api.EPI_SWIGLU_BF16,
-                     row_token=r.row_token, row_gate=r.row_gate, out=h)
+                     row_token=r.row_token, row_gate=r.row_gate, out=h, amax_out=h_amax)
     y = torch.zeros(T, N, dtype=torch.float32, device=cuda)
     api.grouped_gemm(xq.codes, xq.scales, xq.s_t, r.m_pad_max, c_w, sf_w, s_w, N, K, E, r.offsets,
                      rac_ld=rac_ld, rho=xq.r_sel, w_sel=w_sel, epilogue=api.EPI_SCATTER_ADD_F32,
@@ -115,6 +116,16 @@ def test_gemm_swiglu_and_scatter(cuda):
     assert np.all(hg[pad] == 0), "padding rows of h must be zero"
     want_y = np.stack([sum(gate[t, j] * ys[(t, j)] for j in range(kr)) for t in range(T)])
     assert rel_fro(y.cpu().numpy(), want_y) <= TOL
+    # the epilogue's max |h| is exactly the amax of the rows it wrote, and
+    # quantizing h with it gives the same result as with the amax pass
+    n_valid = int(off[-1])
+    assert h_amax.item() == h[:n_valid].float().abs().max().item()
+    mv = r.offsets[E:]
+    q1 = api.quantize(h, rac_k=16, m_valid=mv, m_out=r.m_pad_max)
+    q2 = api.quantize(h, rac_k=16, m_valid=mv, m_out=r.m_pad_max, amax=h_amax)
+    torch.cuda.synchronize()
+    assert q1.s_t.item() == q2.s_t.item()
+    assert torch.equal(q1.codes[:n_valid], q2.codes[:n_valid]) and torch.equal(q1.sel, q2.sel)
 
 
 def test_dense_layer_config(cuda):

@@ -25,7 +25,7 @@ def _noalloc(x, rac_k, rac_ld, dev):
                         sel=torch.empty(rac_k, dtype=torch.int32, device=dev),
                         r_sel=torch.empty(M, rac_ld, dtype=torch.bfloat16, device=dev))
     p = api._p
-    st = lib.nvfp4_quantize_noalloc(p(x), M, K, x.stride(0), None, None, p(out.s_t), None, 1, M, p(out.codes),
+    st = lib.nvfp4_quantize_noalloc(p(x), M, K, x.stride(0), None, None, None, p(out.s_t), None, 1, M, p(out.codes),
                                     p(out.scales), p(out.score), rac_k, rac_ld, p(out.sel), p(out.r_sel), None,
                                     api._stream(dev))
     _lib.check(st)
