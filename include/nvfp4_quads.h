@@ -209,21 +209,23 @@ NVFP4_API nvfp4_status nvfp4_qdq_weights(const void *w_dev, int64_t G, int64_t r
  *   topk_idx_dev int32 [T x k_r]: experts by descending logit (equal logits:
  *                lower expert first).
  *   topk_gate_dev float32 [T x k_r]: softmax over the k_r selected logits.
+ *   seg_align    128 or 256: every expert segment is padded to a multiple of
+ *                this many rows (the grouped GEMM's tile height: 256 selects
+ *                its 2-SM shape).
  *   offsets_dev  int32 [E+1]: expert e owns routed rows
- *                [offsets[e], offsets[e+1]); every segment is padded to a
- *                multiple of 128 rows; offsets[E] = total padded rows.
+ *                [offsets[e], offsets[e+1]); offsets[E] = total padded rows.
  *   dst_row_dev  int32 [T x k_r]: routed row of (token t, slot j).  Inside
  *                an expert's segment tokens appear in ascending order.
  *   row_token_dev int32 [M_pad_max]: token of each routed row, -1 for padding
  *                and for rows >= offsets[E].
  *   row_gate_dev float32 [M_pad_max]: gate of each routed row (0 for padding).
- *   M_pad_max    >= T*k_r + E*127 rounded up to 128.
+ *   M_pad_max    >= T*k_r + E*(seg_align-1) rounded up to seg_align.
  * -------------------------------------------------------------------------- */
 NVFP4_API size_t moe_route_workspace_size(int64_t T, int32_t E);
 
 NVFP4_API nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E, int32_t k_r,
                        int32_t *topk_idx_dev, float *topk_gate_dev,
-                       int32_t *offsets_dev, int32_t *dst_row_dev,
+                       int32_t seg_align, int32_t *offsets_dev, int32_t *dst_row_dev,
                        int32_t *row_token_dev, float *row_gate_dev, int64_t M_pad_max,
                        void *workspace, size_t workspace_bytes, void *stream);
 
@@ -294,12 +296,15 @@ NVFP4_API nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_d
  *   a_s_t_dev       float32 [1].
  *   b_codes_dev/b_scales_dev  NVFP4 B, E tensors of [N x K] (per-expert
  *                   swizzled scales), b_s_t_dev float32 [E].
- *   offsets_dev     int32 [E+1] from moe_route (multiples of 128).
+ *   offsets_dev     int32 [E+1] from moe_route, multiples of seg_align.
+ *   seg_align       128: one CTA per SM computes 128-row x 256-feature tiles;
+ *                   256: CTA pairs (2-SM tensor-core tiles, cluster launch)
+ *                   compute 256-row x 256-feature tiles.
  *   rac_ld          0 (no RAC) or the row stride of rho / w_sel, % 64 == 0,
  *                   <= 256; rho_dev bf16 [M_pad_max x rac_ld] and
  *                   w_sel_dev bf16 [E x N x rac_ld].
- * Shapes: K % 256 == 0, N % 256 == 0 (SWIGLU: I % 128 == 0), M_pad_max % 128
- * == 0, E <= 256.  Persistent kernel: one CTA per SM.
+ * Shapes: K % 256 == 0, N % 256 == 0 (SWIGLU: I % 128 == 0), M_pad_max a
+ * multiple of seg_align, E <= 256.  Persistent kernel: one CTA per SM.
  * -------------------------------------------------------------------------- */
 typedef enum {
     MOE_EPI_STORE_F32 = 0,
@@ -312,7 +317,7 @@ NVFP4_API nvfp4_status moe_w4a4_grouped_gemm_rac(
     int64_t M_pad_max,
     const uint8_t *b_codes_dev, const uint8_t *b_scales_dev, const float *b_s_t_dev,
     int64_t N, int64_t K, int32_t E,
-    const int32_t *offsets_dev,
+    const int32_t *offsets_dev, int32_t seg_align,
     int32_t rac_ld, const void *rho_dev, const void *w_sel_dev,
     int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev,
     void *out_dev, int64_t ld_out, float *amax_out_dev,

@@ -33,7 +33,7 @@ SIGNATURES = {
     "nvfp4_qdq_weights": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
                                     c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_route_workspace_size": (c_size_t, [c_int64, c_int32]),
-    "moe_route": (c_int32, [c_void_p, c_int64, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
+    "moe_route": (c_int32, [c_void_p, c_int64, c_int32, c_int32, c_void_p, c_void_p, c_int32, c_void_p, c_void_p,
                             c_void_p, c_void_p, c_int64, c_void_p, c_size_t, c_void_p]),
     "nvfp4_gather_weight_channels": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int64, c_void_p,
                                                c_int32, c_int32, c_void_p, c_void_p]),
@@ -42,7 +42,7 @@ SIGNATURES = {
     "nvfp4_gather_weight_channels_cm": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int64, c_void_p,
                                                   c_int32, c_int32, c_void_p, c_void_p]),
     "moe_w4a4_grouped_gemm_rac": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
-                                            c_void_p, c_int64, c_int64, c_int32, c_void_p, c_int32, c_void_p,
+                                            c_void_p, c_int64, c_int64, c_int32, c_void_p, c_int32, c_int32, c_void_p,
                                             c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_void_p,
                                             c_void_p, c_void_p]),
     "nvfp4_debug_encode": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),

@@ -114,25 +114,26 @@ class Routing:
     row_token: torch.Tensor     # int32 [M_pad_max]
     row_gate: torch.Tensor      # float32 [M_pad_max]
     m_pad_max: int
+    seg_align: int = 128
 
 
-def padded_rows_bound(T: int, k_r: int, E: int) -> int:
-    return -(-(T * k_r + E * 127) // 128) * 128
+def padded_rows_bound(T: int, k_r: int, E: int, seg_align: int = 128) -> int:
+    return -(-(T * k_r + E * (seg_align - 1)) // seg_align) * seg_align
 
 
-def route(logits: torch.Tensor, k_r: int, m_pad_max: int | None = None) -> Routing:
+def route(logits: torch.Tensor, k_r: int, m_pad_max: int | None = None, seg_align: int = 128) -> Routing:
     lib = _lib.load()
     assert logits.dtype == F32 and logits.is_contiguous()
     T, E = logits.shape
     dev = logits.device
     if m_pad_max is None:
-        m_pad_max = padded_rows_bound(T, k_r, E)
+        m_pad_max = padded_rows_bound(T, k_r, E, seg_align)
     r = Routing(torch.empty(T, k_r, dtype=I32, device=dev), torch.empty(T, k_r, dtype=F32, device=dev),
                 torch.empty(E + 1, dtype=I32, device=dev), torch.empty(T, k_r, dtype=I32, device=dev),
                 torch.empty(m_pad_max, dtype=I32, device=dev), torch.empty(m_pad_max, dtype=F32, device=dev),
-                m_pad_max)
+                m_pad_max, seg_align)
     ws = _ws(lib.moe_route_workspace_size(T, E), dev)
-    check(lib.moe_route(_p(logits), T, E, k_r, _p(r.topk_idx), _p(r.topk_gate), _p(r.offsets), _p(r.dst_row),
+    check(lib.moe_route(_p(logits), T, E, k_r, _p(r.topk_idx), _p(r.topk_gate), seg_align, _p(r.offsets), _p(r.dst_row),
                         _p(r.row_token), _p(r.row_gate), m_pad_max, _p(ws), ws.numel(), _stream(dev)))
     return r
 
@@ -170,14 +171,14 @@ def gather_weight_channels_cm(codes_cm: torch.Tensor, scales_cm: torch.Tensor, N
 
 
 def grouped_gemm(a_codes, a_scales, a_s_t, m_pad_max, b_codes, b_scales, b_s_t, N, K, E, offsets, *,
-                 rac_ld=0, rho=None, w_sel=None, epilogue=EPI_STORE_F32, row_token=None, row_gate=None,
+                 seg_align=128, rac_ld=0, rho=None, w_sel=None, epilogue=EPI_STORE_F32, row_token=None, row_gate=None,
                  out=None, ld_out=None, amax_out=None, dev_status=None):
     """moe_w4a4_grouped_gemm_rac (see the header)."""
     lib = _lib.load()
     if ld_out is None:
         ld_out = out.stride(0)
     check(lib.moe_w4a4_grouped_gemm_rac(_p(a_codes), _p(a_scales), _p(a_s_t), m_pad_max, _p(b_codes),
-                                        _p(b_scales), _p(b_s_t), N, K, E, _p(offsets), rac_ld, _p(rho),
+                                        _p(b_scales), _p(b_s_t), N, K, E, _p(offsets), seg_align, rac_ld, _p(rho),
                                         _p(w_sel), epilogue, _p(row_token), _p(row_gate), _p(out), ld_out,
                                         _p(amax_out), _p(dev_status), _stream(out.device)))
     return out

@@ -1,39 +1,57 @@
 // gemm.cu -- persistent grouped W4A4 (NVFP4) expert GEMM with Residual
 // Activation Compensation on the sm_100a tensor cores.
 //
-// One CTA per SM, 10 warps:
-//   warp 0      TMA producer (one lane): per 256-element K step it loads the
-//               A tile (128 rows x 128 B of packed E2M1), the B tile (two
-//               128-row boxes), and the matching 512-byte scale atoms (bulk
-//               copies) into a 4-stage shared-memory ring; then the RAC
-//               stages (bf16 rho and w_sel tiles, 64 channels each).
-//   warp 1      MMA issuer (one lane): copies the stage's scale atoms to TMEM
-//               (tcgen05.cp 32x128b.warpx4) and issues 4 block-scaled
-//               tcgen05.mma kind::mxf4nvf4 (M128 N256 K64) per stage into one
-//               TMEM accumulator; after the FP4 K loop it drains (commit +
+// Two shapes of the same kernel:
+//   single  one CTA per SM computes 128 routed rows x 256 output features;
+//           expert segments padded to 128 rows.
+//   pair    a 2-CTA cluster (tcgen05 .cta_group::2) computes 256 routed rows
+//           x 256 features: each CTA holds 128 rows of A, half of B (128
+//           features) and the scale factors its half needs; the even CTA
+//           ("leader") issues every scale-factor copy and MMA for both SMs.
+//           Each scale copy and each MMA then covers twice the work, and each
+//           SM stages half the B bytes.  Expert segments padded to 256 rows.
+//
+// Warps (352 threads per CTA):
+//   warp 0      TMA producer (one lane): per 256-element K step the A tile
+//               (128 rows x 128 B packed E2M1, 128-byte swizzle), this CTA's B
+//               tile(s) and the 512-byte scale atoms, into a ring of stages;
+//               then the RAC stages (bf16 rho and w_sel tiles, 64 channels).
+//               In the pair shape both CTAs load their halves and every copy
+//               completes on the leader's barrier.
+//   warp 10     scale-factor copier (one lane, leader only in the pair shape):
+//               once a stage has landed, copies its 12 scale atoms into that
+//               stage's own TMEM scale buffer (tcgen05.cp 32x128b.warpx4) and
+//               commits to the stage's sf_full barrier.  Issued from their own
+//               thread, the copies overlap the MMAs of earlier stages; issued
+//               from the MMA thread they would serialize with them (12 copies
+//               cost about as much tensor-pipe time as the stage's 4 MMAs).
+//               A stage's buffer is free again when the stage is: the
+//               producer refills a stage only after the MMAs reading it are
+//               done.
+//   warp 1      MMA issuer (one lane, leader only in the pair shape): per
+//               stage 4 block-scaled tcgen05.mma kind::mxf4nvf4 (K64) into
+//               one TMEM accumulator; after the FP4 K loop it drains (commit +
 //               wait) and accumulates the RAC stages with kind::f16 BF16 MMAs
-//               (M128 N256 K16) into the same accumulator.
+//               (K16) into the same accumulator.
 //   warps 2..9  epilogue: each warp copies its TMEM slice (32-lane quadrant
 //               w % 4, one half of the columns) into registers and releases
 //               the accumulator at once, so the next tile's MMAs overlap the
 //               math and stores: y = s_a s_b D, then store f32 / SwiGLU ->
-//               bf16 / router-weighted atomic scatter-add into the token-major
+//               bf16 / router-weighted scatter-add into the token-major
 //               output.
-// Tiles: 128 routed rows x 256 output features (SwiGLU: 128 gate + the 128
-// matching up features).  Every expert's routed-row segment is a multiple of
-// 128, so a tile never spans two experts; the tile count comes from the
-// device-side offsets (no host synchronization).
+// Tiles never span two experts (segments are multiples of the tile height);
+// the tile count comes from the device-side offsets (no host sync).
 //
-// Shared memory: a 4-stage ring of 54 KB stages for the SwiGLU (bf16) epilogue;
-// the f32 epilogues use 3 stages and a 34 KB staging area from which each lane
+// Shared memory: a ring of stages (single 54 KB, pair 38 KB); the f32
+// epilogues give up one stage for a 34 KB staging area from which each lane
 // writes 64 contiguous floats of its row with one 256-byte bulk store or bulk
-// add-reduction (cp.reduce.async.bulk .add.f32) -- full-line traffic instead
-// of per-thread 16-byte stores or atomics.
-// TMEM: 512 columns = accumulator [0,256) + scale factors of A [256,272)
-// (4 atoms x 4 columns) + scale factors of B [272,304) (4 x 8 columns).
+// add-reduction (cp.reduce.async.bulk .add.f32).
+// TMEM: 512 columns = accumulator [0,256) + one 48-column scale buffer per
+// stage at 256 + 48 s: A's scale factors in its first 16 columns (4 atoms x 4
+// columns), B's in the next 32 (4 x 8 columns); at most 5 stages.
 // Every mbarrier wait is bounded (1 s); on expiry the kernel records
 // NVFP4_ERR_TIMEOUT, all roles stop, in-flight copies and MMAs are drained
-// (bounded) and TMEM is freed before exit.
+// (bounded) and TMEM is freed before exit.  No TMA load uses multicast.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -44,32 +62,37 @@
 namespace nvfp4 {
 namespace gemm {
 
-constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int MAX_STAGES = 4;
-constexpr uint32_t A_BYTES = BM * 128;          // 16 KB
-constexpr uint32_t B_BYTES = BN * 128;          // 32 KB
+constexpr int MAX_STAGES = 5;
+constexpr uint32_t A_BYTES = 128 * 128;         // 16 KB: 128 rows x 256 FP4
 constexpr uint32_t SFA_BYTES = 4 * 512;         // 4 atoms (K=256 / 64)
-constexpr uint32_t SFB_BYTES = 8 * 512;         // 2 row blocks x 4 atoms
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr uint32_t RAC_STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 320;           // producer, MMA, 8 epilogue warps
+constexpr uint32_t SFB_BYTES = 8 * 512;         // 2 row blocks x 4 atoms (all 256 features)
+constexpr int NUM_THREADS = 352;                // producer, MMA, 8 epilogue warps, scale copier
 constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
+constexpr uint32_t ACC_COL = 0, SF_COL = 256, SF_STRIDE = 48;  // scale buffer of stage s: SF_COL + 48 s
+constexpr int COPY_WARP = 10;
 constexpr int MAX_E = 256;
 constexpr uint64_t TIMEOUT_NS = 1000000000ull;
-// f32 epilogues stage rows in shared memory and write them with 256-byte bulk
-// copies / bulk add-reductions: per epilogue warp 16 row slots of 64 floats,
-// padded to 68 floats so the 16 writing lanes spread over the banks.
-constexpr uint32_t SLOT_FLOATS = 68;
+constexpr uint32_t SLOT_FLOATS = 68;            // 64 floats + 4 padding (bank spread)
 constexpr uint32_t STAGING_BYTES = EPI_WARPS * 16 * SLOT_FLOATS * 4;
 
-template <int STAGES>
+template <bool PAIR>
+struct Geo {
+    static constexpr int TILE_M = PAIR ? 256 : 128;                        // routed rows per tile
+    static constexpr uint32_t B_LOCAL = (PAIR ? 128 : 256) * 128;           // B bytes this CTA stages
+    static constexpr uint32_t STAGE = A_BYTES + B_LOCAL + SFA_BYTES + SFB_BYTES;
+    static constexpr uint32_t RAC_STAGE = A_BYTES + B_LOCAL;
+    static constexpr uint32_t TX = (PAIR ? 2 : 1) * STAGE;                  // bytes the full barrier expects
+    static constexpr uint32_t RAC_TX = (PAIR ? 2 : 1) * RAC_STAGE;
+};
+
+template <int STAGES, bool PAIR, bool STAGING>
 struct Cfg {
-    static constexpr bool STAGING = STAGES < MAX_STAGES;      // f32 epilogues give up one stage for staging
-    static constexpr uint32_t SMEM = STAGES * STAGE_BYTES + (STAGING ? STAGING_BYTES : 0) + 1024 /*align*/ +
-                                     2048 /*barriers, offsets*/;
+    static constexpr uint32_t SMEM = STAGES * Geo<PAIR>::STAGE + (STAGING ? STAGING_BYTES : 0) +
+                                     1024 /*align*/ + 2048 /*barriers, offsets*/;
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(SF_COL + SF_STRIDE * STAGES <= TMEM_COLS, "TMEM budget");
 };
 
 struct Params {
@@ -93,10 +116,12 @@ struct Params {
 
 struct Shared {
     uint64_t full[MAX_STAGES];
+    uint64_t sf_full[MAX_STAGES];
     uint64_t empty[MAX_STAGES];
     uint64_t tmem_full;
     uint64_t tmem_empty;
     uint64_t drain;
+    uint64_t cp_drain;
     uint32_t tmem_base;
     int abort_flag;
     int offsets[MAX_E + 1];
@@ -134,46 +159,62 @@ __device__ __forceinline__ int find_expert(const int *off, int E, int m0)
 
 __device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
-template <int STAGES>
+// Scale-atom row of the 2D [bytes/256 x 256] view of a scale buffer.
+__device__ __forceinline__ int32_t sf_row(int64_t byte_off) { return (int32_t)(byte_off >> 8); }
+
+template <int STAGES, bool PAIR, bool STAGING>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-           const __grid_constant__ CUtensorMap tm_ra, const __grid_constant__ CUtensorMap tm_rb, Params p)
+           const __grid_constant__ CUtensorMap tm_ra, const __grid_constant__ CUtensorMap tm_rb,
+           const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb, Params p)
 {
+    using G = Geo<PAIR>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *stage_base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *staging = reinterpret_cast<float *>(stage_base + STAGES * STAGE_BYTES);
-    Shared *sh = reinterpret_cast<Shared *>(stage_base + STAGES * STAGE_BYTES +
-                                            (Cfg<STAGES>::STAGING ? STAGING_BYTES : 0));
+    float *staging = reinterpret_cast<float *>(stage_base + STAGES * G::STAGE);
+    Shared *sh = reinterpret_cast<Shared *>(stage_base + STAGES * G::STAGE + (STAGING ? STAGING_BYTES : 0));
     volatile int *abort_flag = &sh->abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
+    const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;       // 0 = leader
+    const bool leader = rank == 0;
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;   // tile-scheduling unit
+    const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             ptx::mbar_init(ptx::smem_u32(&sh->full[s]), 1);
+            ptx::mbar_init(ptx::smem_u32(&sh->sf_full[s]), 1);
             ptx::mbar_init(ptx::smem_u32(&sh->empty[s]), 1);
         }
         ptx::mbar_init(ptx::smem_u32(&sh->tmem_full), 1);
-        ptx::mbar_init(ptx::smem_u32(&sh->tmem_empty), EPI_WARPS);
+        ptx::mbar_init(ptx::smem_u32(&sh->tmem_empty), PAIR ? 2 * EPI_WARPS : EPI_WARPS);
         ptx::mbar_init(ptx::smem_u32(&sh->drain), 1);
+        ptx::mbar_init(ptx::smem_u32(&sh->cp_drain), 1);
         sh->abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
     }
     for (int i = threadIdx.x; i <= E; i += NUM_THREADS) sh->offsets[i] = p.offsets[i];
     if (warp == 0) {
-        ptx::tmem_alloc(ptx::smem_u32(&sh->tmem_base), TMEM_COLS);
-        ptx::tmem_relinquish();
+        if (PAIR) {
+            ptx::tmem_alloc_pair(ptx::smem_u32(&sh->tmem_base), TMEM_COLS);
+            ptx::tmem_relinquish_pair();
+        } else {
+            ptx::tmem_alloc(ptx::smem_u32(&sh->tmem_base), TMEM_COLS);
+            ptx::tmem_relinquish();
+        }
     }
     ptx::tc_fence_before();
-    __syncthreads();
+    if (PAIR) ptx::cluster_sync();         // barriers of both CTAs initialized before any remote use
+    else __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
 
     const int swiglu = p.epilogue == MOE_EPI_SWIGLU_BF16;
     const int n_tiles = swiglu ? p.inter / 128 : (int)(p.N / BN);
-    const int m_tiles = sh->offsets[E] / BM;
+    const int m_tiles = sh->offsets[E] / G::TILE_M;
     const int total = m_tiles * n_tiles;
     const int nkb = (int)(p.K / 256);
     const int nrk = p.rac_ld / 64;
@@ -189,42 +230,63 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             bool issued[STAGES];
             for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_phase[s] = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+            for (int t = unit; ok && t < total; t += n_units) {
                 const int mt = t / n_tiles, nt = t % n_tiles;
-                const int m0 = mt * BM;
+                const int m0 = mt * G::TILE_M;
                 const int e = find_expert(sh->offsets, E, m0);
-                int nrow0, nrow1;  // rows inside expert e's [N x K] weight
+                const int arow = m0 + (int)rank * 128;      // this CTA's 128 rows of A
+                int nrow0, nrow1;  // rows inside expert e's [N x K] weight (the two 128-feature halves)
                 if (swiglu) { nrow0 = nt * 128; nrow1 = p.inter + nt * 128; }
                 else { nrow0 = nt * BN; nrow1 = nt * BN + 128; }
                 const int brow0 = (int)(e * p.N) + nrow0, brow1 = (int)(e * p.N) + nrow1;
-                const uint8_t *sfa_src = p.a_scales + (int64_t)(m0 / 128) * (p.K / 64) * 512;
-                const uint8_t *sfb_e = p.b_scales + (int64_t)e * sf_per_expert;
-                const uint8_t *sfb_src0 = sfb_e + (int64_t)(nrow0 / 128) * (p.K / 64) * 512;
-                const uint8_t *sfb_src1 = sfb_e + (int64_t)(nrow1 / 128) * (p.K / 64) * 512;
+                const int64_t sfa_off = (int64_t)(arow / 128) * (p.K / 64) * 512;
+                const int64_t sfb_e = (int64_t)e * sf_per_expert;
+                const int64_t sfb_off0 = sfb_e + (int64_t)(nrow0 / 128) * (p.K / 64) * 512;
+                const int64_t sfb_off1 = sfb_e + (int64_t)(nrow1 / 128) * (p.K / 64) * 512;
                 for (int kb = 0; kb < nkb + nrk; ++kb) {
                     if (!wait_bar(ptx::smem_u32(&sh->empty[stage]), phase ^ 1u, abort_flag, p.dev_status)) {
                         ok = false;
                         break;
                     }
-                    uint8_t *sa = stage_base + stage * STAGE_BYTES;
+                    uint8_t *sa = stage_base + stage * G::STAGE;
                     uint8_t *sb = sa + A_BYTES;
                     const uint32_t fb = ptx::smem_u32(&sh->full[stage]);
-                    if (kb < nkb) {
-                        uint8_t *ssfa = sb + B_BYTES;
+                    if (PAIR) {
+                        const uint32_t lfb = ptx::mapa_shared(fb, 0);     // the leader's barrier
+                        const int browr = rank ? brow1 : brow0;
+                        if (kb < nkb) {
+                            uint8_t *ssfa = sb + G::B_LOCAL;
+                            uint8_t *ssfb = ssfa + SFA_BYTES;
+                            if (leader) ptx::mbar_arrive_expect_tx(fb, G::TX);
+                            ptx::tma_load_2d_pair(ptx::smem_u32(sa), &tm_a, kb * 128, arow, lfb);
+                            ptx::tma_load_2d_pair(ptx::smem_u32(sb), &tm_b, kb * 128, browr, lfb);
+                            ptx::tma_load_2d_pair(ptx::smem_u32(ssfa), &tm_sfa, 0, sf_row(sfa_off + kb * 2048), lfb);
+                            ptx::tma_load_2d_pair(ptx::smem_u32(ssfb), &tm_sfb, 0, sf_row(sfb_off0 + kb * 2048), lfb);
+                            ptx::tma_load_2d_pair(ptx::smem_u32(ssfb + SFB_BYTES / 2), &tm_sfb, 0,
+                                                  sf_row(sfb_off1 + kb * 2048), lfb);
+                        } else {
+                            const int rk = kb - nkb;
+                            if (leader) ptx::mbar_arrive_expect_tx(fb, G::RAC_TX);
+                            ptx::tma_load_2d_pair(ptx::smem_u32(sa), &tm_ra, rk * 64, arow, lfb);
+                            ptx::tma_load_2d_pair(ptx::smem_u32(sb), &tm_rb, rk * 64, browr, lfb);
+                        }
+                    } else if (kb < nkb) {
+                        uint8_t *ssfa = sb + G::B_LOCAL;
                         uint8_t *ssfb = ssfa + SFA_BYTES;
-                        ptx::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                        ptx::mbar_arrive_expect_tx(fb, G::TX);
                         ptx::tma_load_2d(ptx::smem_u32(sa), &tm_a, kb * 128, m0, fb);
                         ptx::tma_load_2d(ptx::smem_u32(sb), &tm_b, kb * 128, brow0, fb);
-                        ptx::tma_load_2d(ptx::smem_u32(sb + B_BYTES / 2), &tm_b, kb * 128, brow1, fb);
-                        ptx::bulk_load(ptx::smem_u32(ssfa), sfa_src + kb * 2048, SFA_BYTES, fb);
-                        ptx::bulk_load(ptx::smem_u32(ssfb), sfb_src0 + kb * 2048, SFB_BYTES / 2, fb);
-                        ptx::bulk_load(ptx::smem_u32(ssfb + SFB_BYTES / 2), sfb_src1 + kb * 2048, SFB_BYTES / 2, fb);
+                        ptx::tma_load_2d(ptx::smem_u32(sb + G::B_LOCAL / 2), &tm_b, kb * 128, brow1, fb);
+                        ptx::bulk_load(ptx::smem_u32(ssfa), p.a_scales + sfa_off + kb * 2048, SFA_BYTES, fb);
+                        ptx::bulk_load(ptx::smem_u32(ssfb), p.b_scales + sfb_off0 + kb * 2048, SFB_BYTES / 2, fb);
+                        ptx::bulk_load(ptx::smem_u32(ssfb + SFB_BYTES / 2), p.b_scales + sfb_off1 + kb * 2048,
+                                       SFB_BYTES / 2, fb);
                     } else {
                         const int rk = kb - nkb;
-                        ptx::mbar_arrive_expect_tx(fb, RAC_STAGE_BYTES);
+                        ptx::mbar_arrive_expect_tx(fb, G::RAC_TX);
                         ptx::tma_load_2d(ptx::smem_u32(sa), &tm_ra, rk * 64, m0, fb);
                         ptx::tma_load_2d(ptx::smem_u32(sb), &tm_rb, rk * 64, brow0, fb);
-                        ptx::tma_load_2d(ptx::smem_u32(sb + B_BYTES / 2), &tm_rb, rk * 64, brow1, fb);
+                        ptx::tma_load_2d(ptx::smem_u32(sb + G::B_LOCAL / 2), &tm_rb, rk * 64, brow1, fb);
                     }
                     issued[stage] = true;
                     issued_phase[stage] = phase;
@@ -233,80 +295,148 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             }
             if (!ok) {
                 // drain copies still in flight before the CTA's memory is released
-                for (int s = 0; s < STAGES; ++s)
-                    if (issued[s])
-                        wait_bar(ptx::smem_u32(&sh->full[s]), issued_phase[s], abort_flag, p.dev_status, true);
+                if (!PAIR || leader) {
+                    for (int s = 0; s < STAGES; ++s)
+                        if (issued[s])
+                            wait_bar(ptx::smem_u32(&sh->full[s]), issued_phase[s], abort_flag, p.dev_status, true);
+                } else {
+                    // the peer's copies complete on the leader's barriers: give them 100 us
+                    const uint64_t t0 = globaltimer_ns();
+                    while (globaltimer_ns() - t0 < 100000ull) { }
+                }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             // --------------------------------------------------- MMA issuer
-            const uint32_t idesc4 = ptx::idesc_mxf4nvf4(BM, BN);
-            const uint32_t idesc16 = ptx::idesc_bf16(BM, BN);
+            const uint32_t idesc4 = ptx::idesc_mxf4nvf4(PAIR ? 256 : 128, BN);
+            const uint32_t idesc16 = ptx::idesc_bf16(PAIR ? 256 : 128, BN);
             uint32_t stage = 0, phase = 0, drain_phase = 0;
             bool ok = true;
             bool issued_any = false;
             int iter = 0;
-            for (int t = blockIdx.x; ok && t < total; t += gridDim.x, ++iter) {
+            for (int t = unit; ok && t < total; t += n_units, ++iter) {
                 if (!wait_bar(ptx::smem_u32(&sh->tmem_empty), (uint32_t)(iter & 1) ^ 1u, abort_flag, p.dev_status)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
                 for (int kb = 0; kb < nkb && ok; ++kb) {
-                    if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t sa = ptx::smem_u32(stage_base + stage * STAGE_BYTES);
-                    const uint32_t sb = sa + A_BYTES;
-                    const uint32_t ssfa = sb + B_BYTES;
-                    const uint32_t ssfb = ssfa + SFA_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        ptx::tmem_cp_32x128b_warpx4(tmem + SFA_COL + 4 * kk, ptx::make_sdesc(ssfa + 512 * kk, 0, 128, 0));
-                        ptx::tmem_cp_32x128b_warpx4(tmem + SFB_COL + 8 * kk, ptx::make_sdesc(ssfb + 512 * kk, 0, 128, 0));
-                        ptx::tmem_cp_32x128b_warpx4(tmem + SFB_COL + 8 * kk + 4,
-                                                    ptx::make_sdesc(ssfb + SFB_BYTES / 2 + 512 * kk, 0, 128, 0));
+                    // the stage's data has landed and its scale factors are in TMEM
+                    if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status) ||
+                        !wait_bar(ptx::smem_u32(&sh->sf_full[stage]), phase, abort_flag, p.dev_status)) {
+                        ok = false;
+                        break;
                     }
+                    ptx::tc_fence_after();
+                    const uint32_t sa = ptx::smem_u32(stage_base + stage * G::STAGE);
+                    const uint32_t sb = sa + A_BYTES;
+                    const uint32_t sfa = tmem + SF_COL + SF_STRIDE * stage, sfb = sfa + 16;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         uint64_t ad = ptx::make_sdesc(sa + 32 * kk, 16, 1024, 2);
                         uint64_t bd = ptx::make_sdesc(sb + 32 * kk, 16, 1024, 2);
-                        ptx::mma_mxf4nvf4(tmem + ACC_COL, ad, bd, idesc4, tmem + SFA_COL + 4 * kk,
-                                          tmem + SFB_COL + 8 * kk, (kb | kk) != 0);
+                        if (PAIR)
+                            ptx::mma_mxf4nvf4_pair(tmem + ACC_COL, ad, bd, idesc4, sfa + 4 * kk, sfb + 8 * kk,
+                                                   (kb | kk) != 0);
+                        else
+                            ptx::mma_mxf4nvf4(tmem + ACC_COL, ad, bd, idesc4, sfa + 4 * kk, sfb + 8 * kk,
+                                              (kb | kk) != 0);
                     }
-                    ptx::tc_commit(ptx::smem_u32(&sh->empty[stage]));
+                    if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->empty[stage]), 3);
+                    else ptx::tc_commit(ptx::smem_u32(&sh->empty[stage]));
                     issued_any = true;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (ok && nrk > 0) {
                     // the BF16 MMAs accumulate into the same TMEM tile: wait for
                     // the FP4 MMAs to complete first
-                    ptx::tc_commit(ptx::smem_u32(&sh->drain));
+                    if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->drain), 1);
+                    else ptx::tc_commit(ptx::smem_u32(&sh->drain));
                     if (!wait_bar(ptx::smem_u32(&sh->drain), drain_phase, abort_flag, p.dev_status)) { ok = false; }
                     drain_phase ^= 1u;
                     ptx::tc_fence_after();
                     for (int rk = 0; rk < nrk && ok; ++rk) {
-                        if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status)) { ok = false; break; }
+                        if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status) ||
+                            !wait_bar(ptx::smem_u32(&sh->sf_full[stage]), phase, abort_flag, p.dev_status)) {
+                            ok = false;
+                            break;
+                        }
                         ptx::tc_fence_after();
-                        const uint32_t sa = ptx::smem_u32(stage_base + stage * STAGE_BYTES);
+                        const uint32_t sa = ptx::smem_u32(stage_base + stage * G::STAGE);
                         const uint32_t sb = sa + A_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             uint64_t ad = ptx::make_sdesc(sa + 32 * kk, 16, 1024, 2);
                             uint64_t bd = ptx::make_sdesc(sb + 32 * kk, 16, 1024, 2);
-                            ptx::mma_bf16(tmem + ACC_COL, ad, bd, idesc16, 1u);
+                            if (PAIR) ptx::mma_bf16_pair(tmem + ACC_COL, ad, bd, idesc16, 1u);
+                            else ptx::mma_bf16(tmem + ACC_COL, ad, bd, idesc16, 1u);
                         }
-                        ptx::tc_commit(ptx::smem_u32(&sh->empty[stage]));
+                        if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->empty[stage]), 3);
+                        else ptx::tc_commit(ptx::smem_u32(&sh->empty[stage]));
                         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     }
                 }
-                if (ok) ptx::tc_commit(ptx::smem_u32(&sh->tmem_full));
+                if (ok) {
+                    if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->tmem_full), 3);
+                    else ptx::tc_commit(ptx::smem_u32(&sh->tmem_full));
+                }
             }
             if (!ok && issued_any) {
                 // let every issued MMA finish before TMEM is released
-                ptx::tc_commit(ptx::smem_u32(&sh->drain));
+                if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->drain), 1);
+                else ptx::tc_commit(ptx::smem_u32(&sh->drain));
                 wait_bar(ptx::smem_u32(&sh->drain), drain_phase, abort_flag, p.dev_status, true);
+            }
+        }
+        __syncwarp();
+    } else if (warp == COPY_WARP) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------- scale-factor copier
+            // Follows the producer's stage sequence; per stage one commit to
+            // sf_full (RAC stages carry no scale factors: an empty commit
+            // keeps the barrier's phase in step with full).
+            uint32_t stage = 0, phase = 0;
+            bool ok = true, issued_any = false;
+            for (int t = unit; ok && t < total; t += n_units) {
+                for (int kb = 0; kb < nkb + nrk; ++kb) {
+                    if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    if (kb < nkb) {
+                        const uint32_t ssfa = ptx::smem_u32(stage_base + stage * G::STAGE) + A_BYTES + G::B_LOCAL;
+                        const uint32_t ssfb = ssfa + SFA_BYTES;
+                        const uint32_t sfa = tmem + SF_COL + SF_STRIDE * stage, sfb = sfa + 16;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t da = ptx::make_sdesc(ssfa + 512 * kk, 0, 128, 0);
+                            const uint64_t db0 = ptx::make_sdesc(ssfb + 512 * kk, 0, 128, 0);
+                            const uint64_t db1 = ptx::make_sdesc(ssfb + SFB_BYTES / 2 + 512 * kk, 0, 128, 0);
+                            if (PAIR) {
+                                ptx::tmem_cp_32x128b_warpx4_pair(sfa + 4 * kk, da);
+                                ptx::tmem_cp_32x128b_warpx4_pair(sfb + 8 * kk, db0);
+                                ptx::tmem_cp_32x128b_warpx4_pair(sfb + 8 * kk + 4, db1);
+                            } else {
+                                ptx::tmem_cp_32x128b_warpx4(sfa + 4 * kk, da);
+                                ptx::tmem_cp_32x128b_warpx4(sfb + 8 * kk, db0);
+                                ptx::tmem_cp_32x128b_warpx4(sfb + 8 * kk + 4, db1);
+                            }
+                        }
+                    }
+                    if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->sf_full[stage]), 1);
+                    else ptx::tc_commit(ptx::smem_u32(&sh->sf_full[stage]));
+                    issued_any = true;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok && issued_any) {
+                // copies still in flight complete before TMEM is released
+                if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->cp_drain), 1);
+                else ptx::tc_commit(ptx::smem_u32(&sh->cp_drain));
+                wait_bar(ptx::smem_u32(&sh->cp_drain), 0, abort_flag, p.dev_status, true);
             }
         }
         __syncwarp();
@@ -317,17 +447,19 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
         // accumulator for the next tile's MMAs, then computes and stores.
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
-        const int row_in_tile = q * 32 + lane;
+        const int row_in_tile = (int)rank * 128 + q * 32 + lane;
         const float s_a = *p.a_s_t;
+        const uint32_t empty_bar = PAIR ? ptx::mapa_shared(ptx::smem_u32(&sh->tmem_empty), 0)
+                                        : ptx::smem_u32(&sh->tmem_empty);
         int iter = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++iter) {
+        for (int t = unit; t < total; t += n_units, ++iter) {
             bool ok = true;
             if (lane == 0) ok = wait_bar(ptx::smem_u32(&sh->tmem_full), (uint32_t)(iter & 1), abort_flag, p.dev_status);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
             ptx::tc_fence_after();
             const int mt = t / n_tiles, nt = t % n_tiles;
-            const int m0 = mt * BM;
+            const int m0 = mt * G::TILE_M;
             const int e = find_expert(sh->offsets, E, m0);
             const uint32_t tbase = tmem + ACC_COL + ((uint32_t)(q * 32) << 16);
             uint32_t v[128];
@@ -345,7 +477,10 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             ptx::tmem_ld_wait();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&sh->tmem_empty));
+            if (lane == 0) {
+                if (PAIR) ptx::mbar_arrive_cluster(empty_bar);
+                else ptx::mbar_arrive(empty_bar);
+            }
 
             const float scale = __fmul_rn(s_a, p.b_s_t[e]);
             const int64_t r = (int64_t)m0 + row_in_tile;
@@ -376,7 +511,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                     for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
                     if (lane == 0) atomicMax(p.amax_out, __float_as_uint(hmax));
                 }
-            } else if (Cfg<STAGES>::STAGING) {
+            } else if (STAGING) {
                 // f32 out: each lane stages 64 contiguous floats of its row and
                 // moves them with one 256-byte bulk store / bulk add-reduction;
                 // lanes 0-15 then 16-31 share the warp's 16 slots.
@@ -407,39 +542,56 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                         __syncwarp();
                     }
                 }
-            } else if (p.epilogue == MOE_EPI_STORE_F32) {
-                if (token >= 0) {
-                    float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + r * p.ld_out +
-                                                             nt * BN + half * 128);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        dst[j] = make_float4(scale * __uint_as_float(v[4 * j]), scale * __uint_as_float(v[4 * j + 1]),
-                                             scale * __uint_as_float(v[4 * j + 2]), scale * __uint_as_float(v[4 * j + 3]));
-                }
-            } else if (token >= 0) {
-                const float gw = __fmul_rn(scale, p.row_gate[r]);
-                float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + (int64_t)token * p.ld_out +
-                                                         nt * BN + half * 128);
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    atomicAdd(dst + j, make_float4(gw * __uint_as_float(v[4 * j]), gw * __uint_as_float(v[4 * j + 1]),
-                                                   gw * __uint_as_float(v[4 * j + 2]), gw * __uint_as_float(v[4 * j + 3])));
             }
         }
-        if (Cfg<STAGES>::STAGING) ptx::bulk_wait_all();     // this lane's bulk writes are complete
+        if (STAGING) ptx::bulk_wait_all();     // this lane's bulk writes are complete
     }
 
     ptx::tc_fence_before();
-    __syncthreads();
+    if (PAIR) ptx::cluster_sync();         // neither CTA leaves while the pair still uses its memory
+    else __syncthreads();
     if (warp == 0) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, TMEM_COLS);
+        if (PAIR) ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
+        else ptx::tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
 // ----------------------------------------------------------------- host side
 
-static bool smem_attr_done[2][64];
+template <int STAGES, bool PAIR, bool STAGING>
+static nvfp4_status launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, const CUtensorMap &tm_ra,
+                           const CUtensorMap &tm_rb, const CUtensorMap &tm_sfa, const CUtensorMap &tm_sfb,
+                           const Params &p, int units, cudaStream_t st)
+{
+    static bool attr_done[64];
+    auto kern = k_moe_gemm<STAGES, PAIR, STAGING>;
+    const uint32_t smem = Cfg<STAGES, PAIR, STAGING>::SMEM;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return check_launch("moe_w4a4_grouped_gemm_rac: smem attribute");
+        attr_done[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)(PAIR ? 2 * units : units));
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    if (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    if (cudaLaunchKernelEx(&cfg, kern, tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p) != cudaSuccess)
+        return check_launch("k_moe_gemm");
+    return check_launch("k_moe_gemm");
+}
 
 }  // namespace gemm
 }  // namespace nvfp4
@@ -449,9 +601,9 @@ using namespace nvfp4;
 extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
     const uint8_t *a_codes_dev, const uint8_t *a_scales_dev, const float *a_s_t_dev, int64_t M_pad_max,
     const uint8_t *b_codes_dev, const uint8_t *b_scales_dev, const float *b_s_t_dev, int64_t N, int64_t K, int32_t E,
-    const int32_t *offsets_dev, int32_t rac_ld, const void *rho_dev, const void *w_sel_dev, int32_t epilogue,
-    const int32_t *row_token_dev, const float *row_gate_dev, void *out_dev, int64_t ld_out, float *amax_out_dev,
-    int32_t *dev_status, void *stream)
+    const int32_t *offsets_dev, int32_t seg_align, int32_t rac_ld, const void *rho_dev, const void *w_sel_dev,
+    int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev, void *out_dev, int64_t ld_out,
+    float *amax_out_dev, int32_t *dev_status, void *stream)
 {
     using namespace nvfp4::gemm;
     cudaStream_t st = (cudaStream_t)stream;
@@ -459,6 +611,8 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
                   offsets_dev && row_token_dev && out_dev, NVFP4_ERR_INVALID_ARG,
                   "moe_w4a4_grouped_gemm_rac: null pointer");
     NVFP4_REQUIRE(epilogue >= 0 && epilogue <= 2, NVFP4_ERR_INVALID_ARG, "moe_w4a4_grouped_gemm_rac: bad epilogue");
+    NVFP4_REQUIRE(seg_align == 128 || seg_align == 256, NVFP4_ERR_INVALID_ARG,
+                  "moe_w4a4_grouped_gemm_rac: seg_align must be 128 or 256");
     NVFP4_REQUIRE(epilogue != MOE_EPI_SCATTER_ADD_F32 || row_gate_dev, NVFP4_ERR_INVALID_ARG,
                   "moe_w4a4_grouped_gemm_rac: scatter-add needs row_gate");
     NVFP4_REQUIRE(E >= 1 && E <= MAX_E, NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_w4a4_grouped_gemm_rac: 1 <= E <= 256");
@@ -466,8 +620,9 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
                   "moe_w4a4_grouped_gemm_rac: K must be a positive multiple of 256 (K=%lld)", (long long)K);
     NVFP4_REQUIRE(N >= 256 && N % 256 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
                   "moe_w4a4_grouped_gemm_rac: N must be a positive multiple of 256 (N=%lld)", (long long)N);
-    NVFP4_REQUIRE(M_pad_max >= 128 && M_pad_max % 128 == 0 && M_pad_max < (1ll << 31), NVFP4_ERR_UNSUPPORTED_SHAPE,
-                  "moe_w4a4_grouped_gemm_rac: M_pad_max must be a positive multiple of 128");
+    NVFP4_REQUIRE(M_pad_max >= seg_align && M_pad_max % seg_align == 0 && M_pad_max < (1ll << 31),
+                  NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "moe_w4a4_grouped_gemm_rac: M_pad_max must be a positive multiple of seg_align");
     NVFP4_REQUIRE((int64_t)E * N < (1ll << 31), NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_w4a4_grouped_gemm_rac: E*N too large");
     NVFP4_REQUIRE(rac_ld >= 0 && rac_ld <= 256 && rac_ld % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
                   "moe_w4a4_grouped_gemm_rac: rac_ld must be 0..256 and a multiple of 64");
@@ -486,7 +641,7 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
                   aligned16(b_scales_dev) && aligned16(out_dev) && (rac_ld == 0 || (aligned16(rho_dev) && aligned16(w_sel_dev))),
                   NVFP4_ERR_ALIGNMENT, "moe_w4a4_grouped_gemm_rac: pointers must be 16-byte aligned");
 
-    CUtensorMap tm_a, tm_b, tm_ra, tm_rb;
+    CUtensorMap tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     bool ok = make_tmap_2d(&tm_a, a_codes_dev, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)M_pad_max,
                            (uint64_t)K / 2, 128, 128, sw) &&
@@ -501,19 +656,21 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
         tm_ra = tm_a;
         tm_rb = tm_b;
     }
+    const bool pair = seg_align == 256;
+    if (ok && pair) {
+        // scale buffers viewed as [bytes/256 x 256] for 2 KB (4-atom) TMA boxes
+        const uint64_t sfa_bytes = (uint64_t)M_pad_max * (uint64_t)(K / 16);
+        const uint64_t sfb_bytes = (uint64_t)E * (uint64_t)(((N + 127) / 128) * 128) * (uint64_t)(K / 16);
+        ok = make_tmap_2d(&tm_sfa, a_scales_dev, CU_TENSOR_MAP_DATA_TYPE_UINT8, 256, sfa_bytes / 256, 256, 256, 8,
+                          CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             make_tmap_2d(&tm_sfb, b_scales_dev, CU_TENSOR_MAP_DATA_TYPE_UINT8, 256, sfb_bytes / 256, 256, 256, 8,
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
+    } else {
+        tm_sfa = tm_a;
+        tm_sfb = tm_b;
+    }
     NVFP4_REQUIRE(ok, NVFP4_ERR_CUDA, "moe_w4a4_grouped_gemm_rac: tensor map encoding failed");
 
-    // SwiGLU (bf16 out) keeps 4 stages; the f32 epilogues trade one for staging
-    const bool four = epilogue == MOE_EPI_SWIGLU_BF16;
-    auto kern = four ? k_moe_gemm<4> : k_moe_gemm<3>;
-    const uint32_t smem = four ? Cfg<4>::SMEM : Cfg<3>::SMEM;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !smem_attr_done[four][dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return check_launch("moe_w4a4_grouped_gemm_rac: smem attribute");
-        smem_attr_done[four][dev] = true;
-    }
     Params p{};
     p.a_scales = a_scales_dev;
     p.a_s_t = a_s_t_dev;
@@ -534,9 +691,17 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
     p.dev_status = dev_status;
     if (p.amax_out && cudaMemsetAsync(p.amax_out, 0, sizeof(float), st) != cudaSuccess)
         return check_launch("moe_w4a4_grouped_gemm_rac: memset");
-    int64_t n_tiles = epilogue == MOE_EPI_SWIGLU_BF16 ? inter / 128 : N / BN;
-    int64_t max_tiles = (M_pad_max / BM) * n_tiles;
-    int grid = (int)std::min<int64_t>(num_sms(), max_tiles);
-    kern<<<grid, NUM_THREADS, smem, st>>>(tm_a, tm_b, tm_ra, tm_rb, p);
-    return check_launch("k_moe_gemm");
+    const int64_t n_tiles = epilogue == MOE_EPI_SWIGLU_BF16 ? inter / 128 : N / BN;
+    const int64_t max_tiles = (M_pad_max / seg_align) * n_tiles;
+    const bool swiglu = epilogue == MOE_EPI_SWIGLU_BF16;
+    if (pair) {
+        // SwiGLU (bf16 out): 5 stages; f32 epilogues: 4 stages + staging
+        const int units = (int)std::min<int64_t>(num_sms() / 2, max_tiles);
+        return swiglu ? launch<5, true, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
+                      : launch<4, true, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
+    }
+    // SwiGLU (bf16 out): 4 stages; f32 epilogues: 3 stages + staging
+    const int units = (int)std::min<int64_t>(num_sms(), max_tiles);
+    return swiglu ? launch<4, false, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
+                  : launch<3, false, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
 }

@@ -3,7 +3,8 @@
 //   k_route_topk    one warp per token: k_r rounds of warp argmax over the E
 //                   logits (equal logits: lower expert), softmax over the
 //                   selected logits, per-expert counts (atomics).
-//   k_route_assign  one CTA per expert: padded segment offset from the
+//   k_route_assign  one CTA per expert: padded segment offset (segments are
+//                   multiples of 128 or 256 rows, the GEMM's tile height) from the
 //                   counts, then a block-wide scan over tokens in ascending
 //                   order assigns each (token, slot) routed to the expert its
 //                   row; writes dst_row, row_token, row_gate and the padding.
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ lo
 
 __global__ void __launch_bounds__(1024) k_route_assign(const int32_t *__restrict__ topk_idx,
                                                        const float *__restrict__ topk_gate, int64_t T, int E, int kr,
-                                                       const int32_t *__restrict__ counts,
+                                                       const int32_t *__restrict__ counts, int align,
                                                        int32_t *__restrict__ offsets, int32_t *__restrict__ dst_row,
                                                        int32_t *__restrict__ row_token, float *__restrict__ row_gate)
 {
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(1024) k_route_assign(const int32_t *__restrict
     if (tid == 0) {
         int base = 0, total = 0;
         for (int i = 0; i < E; ++i) {
-            int padded = (counts[i] + 127) / 128 * 128;
+            int padded = (counts[i] + align - 1) / align * align;
             if (i < e) base += padded;
             total += padded;
         }
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(1024) k_route_assign(const int32_t *__restrict
         __syncthreads();
     }
     const int cnt = s_cnt;
-    const int padded = (cnt + 127) / 128 * 128;
+    const int padded = (cnt + align - 1) / align * align;
     for (int i = cnt + tid; i < padded; i += blockDim.x) {
         row_token[base + i] = -1;
         row_gate[base + i] = 0.0f;
@@ -152,7 +153,7 @@ extern "C" size_t moe_route_workspace_size(int64_t T, int32_t E)
 
 extern "C" nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E, int32_t k_r,
                                   int32_t *topk_idx_dev, float *topk_gate_dev,
-                                  int32_t *offsets_dev, int32_t *dst_row_dev,
+                                  int32_t seg_align, int32_t *offsets_dev, int32_t *dst_row_dev,
                                   int32_t *row_token_dev, float *row_gate_dev, int64_t M_pad_max,
                                   void *workspace, size_t workspace_bytes, void *stream)
 {
@@ -161,7 +162,8 @@ extern "C" nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E,
                   row_gate_dev, NVFP4_ERR_INVALID_ARG, "moe_route: null pointer");
     NVFP4_REQUIRE(T >= 0 && E >= 1 && E <= MAX_EXPERTS && k_r >= 1 && k_r <= MAX_TOPK && k_r <= E,
                   NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_route: need 1 <= E <= 256, 1 <= k_r <= min(8, E)");
-    int64_t need_rows = (T * k_r + (int64_t)E * 127 + 127) / 128 * 128;
+    NVFP4_REQUIRE(seg_align == 128 || seg_align == 256, NVFP4_ERR_INVALID_ARG, "moe_route: seg_align must be 128 or 256");
+    int64_t need_rows = (T * k_r + (int64_t)E * (seg_align - 1) + seg_align - 1) / seg_align * seg_align;
     NVFP4_REQUIRE(M_pad_max >= need_rows, NVFP4_ERR_INVALID_ARG,
                   "moe_route: M_pad_max must be >= %lld", (long long)need_rows);
     NVFP4_REQUIRE(M_pad_max < (int64_t)1 << 31, NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_route: too many rows");
@@ -177,7 +179,7 @@ extern "C" nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E,
                                                              counts);
         if (check_launch("k_route_topk") != NVFP4_OK) return NVFP4_ERR_CUDA;
     }
-    k_route_assign<<<(unsigned)E, 1024, 0, st>>>(topk_idx_dev, topk_gate_dev, T, E, k_r, counts, offsets_dev,
+    k_route_assign<<<(unsigned)E, 1024, 0, st>>>(topk_idx_dev, topk_gate_dev, T, E, k_r, counts, seg_align, offsets_dev,
                                                 dst_row_dev, row_token_dev, row_gate_dev);
     return check_launch("k_route_assign");
 }

@@ -28,7 +28,8 @@ from . import api
 
 
 class MoELayerW4A4:
-    def __init__(self, w13: torch.Tensor, w2: torch.Tensor, tokens: int, topk: int, rac_k: int):
+    def __init__(self, w13: torch.Tensor, w2: torch.Tensor, tokens: int, topk: int, rac_k: int,
+                 seg_align: int = 256):
         assert w13.dtype == torch.bfloat16 and w2.dtype == torch.bfloat16
         E, N13, H = w13.shape
         E2, H2, I = w2.shape
@@ -42,7 +43,8 @@ class MoELayerW4A4:
         # channel-major copies: the per-step RAC gathers read only the selected channels
         self.c13_cm, self.sf13_cm = api.weights_channel_major(self.c13, self.sf13, 2 * I, H)
         self.c2_cm, self.sf2_cm = api.weights_channel_major(self.c2, self.sf2, H, I)
-        self.m_pad = api.padded_rows_bound(tokens, topk, E)
+        self.seg_align = seg_align          # 256: 2-SM GEMM tiles; 128: one SM per tile
+        self.m_pad = api.padded_rows_bound(tokens, topk, E, seg_align)
         mp, ld = self.m_pad, max(self.rac_ld, 1)
         self.xq = api.Quantized(
             codes=torch.empty(mp, H // 2, dtype=torch.uint8, device=dev),
@@ -70,7 +72,7 @@ class MoELayerW4A4:
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor) -> torch.Tensor:
         E, H, I, k = self.E, self.H, self.I, self.rac_k
-        r = api.route(logits, self.k_r, self.m_pad) if self.routing is None else self._route_into(logits)
+        r = api.route(logits, self.k_r, self.m_pad, self.seg_align) if self.routing is None else self._route_into(logits)
         self.routing = r
         api.quantize(x, rac_k=k, rac_ld=self.rac_ld, dst_rows=r.dst_row, fanout=self.k_r, m_out=self.m_pad,
                      out=self.xq, workspace=self.ws_x)
@@ -78,7 +80,7 @@ class MoELayerW4A4:
             api.gather_weight_channels_cm(self.c13_cm, self.sf13_cm, 2 * I, H, self.xq.sel, k, self.rac_ld,
                                           out=self.w_sel13)
         api.grouped_gemm(self.xq.codes, self.xq.scales, self.xq.s_t, self.m_pad, self.c13, self.sf13, self.s13,
-                         2 * I, H, E, r.offsets, rac_ld=self.rac_ld if k else 0, rho=self.xq.r_sel,
+                         2 * I, H, E, r.offsets, seg_align=self.seg_align, rac_ld=self.rac_ld if k else 0, rho=self.xq.r_sel,
                          w_sel=self.w_sel13, epilogue=api.EPI_SWIGLU_BF16, row_token=r.row_token,
                          row_gate=r.row_gate, out=self.h, amax_out=self.h_amax)
         api.quantize(self.h, rac_k=k, rac_ld=self.rac_ld, m_out=self.m_pad, m_valid=r.offsets[E:],
@@ -88,7 +90,8 @@ class MoELayerW4A4:
                                           out=self.w_sel2)
         self.y.zero_()
         api.grouped_gemm(self.hq.codes, self.hq.scales, self.hq.s_t, self.m_pad, self.c2, self.sf2, self.s2,
-                         H, I, E, r.offsets, rac_ld=self.rac_ld if k else 0, rho=self.hq.r_sel, w_sel=self.w_sel2,
+                         H, I, E, r.offsets, seg_align=self.seg_align, rac_ld=self.rac_ld if k else 0,
+                         rho=self.hq.r_sel, w_sel=self.w_sel2,
                          epilogue=api.EPI_SCATTER_ADD_F32, row_token=r.row_token, row_gate=r.row_gate, out=self.y)
         return self.y
 
@@ -100,7 +103,7 @@ class MoELayerW4A4:
         if ws is None:
             ws = self._ws_route = api._ws(lib.moe_route_workspace_size(T, E), logits.device)
         api.check(lib.moe_route(api._p(logits), T, E, self.k_r, api._p(r.topk_idx), api._p(r.topk_gate),
-                                api._p(r.offsets), api._p(r.dst_row), api._p(r.row_token), api._p(r.row_gate),
+                                self.seg_align, api._p(r.offsets), api._p(r.dst_row), api._p(r.row_token), api._p(r.row_gate),
                                 r.m_pad_max, api._p(ws), ws.numel(), api._stream(logits.device)))
         return r
 

@@ -66,7 +66,7 @@ def test_argument_errors_are_synchronous():
                             None, fake, 1 << 20, None)
     assert st == 3
     # GEMM shape errors
-    args = [fake, fake, fake, 128, fake, fake, fake, 256, 256, 1, fake, 0, None, None, 0, fake, fake, fake, 256,
+    args = [fake, fake, fake, 128, fake, fake, fake, 256, 256, 1, fake, 128, 0, None, None, 0, fake, fake, fake, 256,
             None, None, None]
     bad_k = list(args)
     bad_k[8] = 320
@@ -75,11 +75,18 @@ def test_argument_errors_are_synchronous():
     bad_e[9] = 300
     assert lib.moe_w4a4_grouped_gemm_rac(*bad_e) == 3
     bad_epi = list(args)
-    bad_epi[14] = 7
+    bad_epi[15] = 7
     assert lib.moe_w4a4_grouped_gemm_rac(*bad_epi) == 1
+    bad_align = list(args)
+    bad_align[11] = 64
+    assert lib.moe_w4a4_grouped_gemm_rac(*bad_align) == 1
+    pair_rows = list(args)
+    pair_rows[11] = 256                      # M_pad_max (128) is not a multiple of 256
+    assert lib.moe_w4a4_grouped_gemm_rac(*pair_rows) == 3
     # routing
-    assert lib.moe_route(fake, 16, 300, 2, fake, fake, fake, fake, fake, fake, 1 << 20, fake, 4096, None) == 3
-    assert lib.moe_route(fake, 16, 8, 2, fake, fake, fake, fake, fake, fake, 128, fake, 4096, None) == 1
+    assert lib.moe_route(fake, 16, 300, 2, fake, fake, 128, fake, fake, fake, fake, 1 << 20, fake, 4096, None) == 3
+    assert lib.moe_route(fake, 16, 8, 2, fake, fake, 128, fake, fake, fake, fake, 128, fake, 4096, None) == 1
+    assert lib.moe_route(fake, 16, 8, 2, fake, fake, 100, fake, fake, fake, fake, 1 << 20, fake, 4096, None) == 1
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

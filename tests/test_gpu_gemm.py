@@ -19,7 +19,7 @@ def gen(rng, shape, scale=1.0):
     return oracle.f32_to_bf16(rng.standard_normal(shape).astype(np.float32) * scale)
 
 
-def _setup(cuda, rng, T, E, kr, N, K, rac_k):
+def _setup(cuda, rng, T, E, kr, N, K, rac_k, align=128):
     x = gen(rng, (T, K))
     ch = rng.choice(K, 4, replace=False)
     xf = oracle.bf16_to_f32(x)
@@ -27,7 +27,7 @@ def _setup(cuda, rng, T, E, kr, N, K, rac_k):
     x = oracle.f32_to_bf16(xf)
     w = gen(rng, (E, N, K), 0.02)
     logits = rng.standard_normal((T, E)).astype(np.float32)
-    r = api.route(torch.from_numpy(logits).to(cuda), kr)
+    r = api.route(torch.from_numpy(logits).to(cuda), kr, seg_align=align)
     rac_ld = -(-rac_k // 64) * 64 if rac_k else 0
     xq = api.quantize(to_bf16_dev(x, cuda), rac_k=rac_k, rac_ld=rac_ld, dst_rows=r.dst_row, fanout=kr,
                       m_out=r.m_pad_max)
@@ -59,6 +59,7 @@ def _oracle_rows(x, w, logits, kr, rac_k, sel):
     return idx, gate, ys
 
 
+@pytest.mark.parametrize("align", [128, 256])
 @pytest.mark.parametrize("T,E,kr,N,K,rac_k", [
     (100, 1, 1, 256, 256, 0),
     (64, 1, 1, 256, 256, 8),
@@ -66,12 +67,12 @@ def _oracle_rows(x, w, logits, kr, rac_k, sel):
     (700, 8, 2, 256, 2048, 32),
     (500, 5, 3, 768, 512, 200),
 ])
-def test_gemm_store_f32(cuda, T, E, kr, N, K, rac_k):
+def test_gemm_store_f32(cuda, T, E, kr, N, K, rac_k, align):
     rng = np.random.default_rng(T + N + K + rac_k)
-    x, w, logits, r, xq, s_w, c_w, sf_w, w_sel, rac_ld = _setup(cuda, rng, T, E, kr, N, K, rac_k)
+    x, w, logits, r, xq, s_w, c_w, sf_w, w_sel, rac_ld = _setup(cuda, rng, T, E, kr, N, K, rac_k, align)
     out = torch.full((r.m_pad_max, N), float("nan"), dtype=torch.float32, device=cuda)
     api.grouped_gemm(xq.codes, xq.scales, xq.s_t, r.m_pad_max, c_w, sf_w, s_w, N, K, E, r.offsets,
-                     rac_ld=rac_ld, rho=xq.r_sel, w_sel=w_sel, epilogue=api.EPI_STORE_F32,
+                     seg_align=align, rac_ld=rac_ld, rho=xq.r_sel, w_sel=w_sel, epilogue=api.EPI_STORE_F32,
                      row_token=r.row_token, row_gate=r.row_gate, out=out)
     torch.cuda.synchronize()
     sel = xq.sel.cpu().numpy() if rac_k else None
@@ -89,19 +90,20 @@ def test_gemm_store_f32(cuda, T, E, kr, N, K, rac_k):
     assert np.all(np.isnan(got[pad]))
 
 
-def test_gemm_swiglu_and_scatter(cuda):
+@pytest.mark.parametrize("align", [128, 256])
+def test_gemm_swiglu_and_scatter(cuda, align):
     rng = np.random.default_rng(11)
     T, E, kr, I, K, rac_k = 400, 6, 2, 256, 512, 32
     N = 2 * I
-    x, w, logits, r, xq, s_w, c_w, sf_w, w_sel, rac_ld = _setup(cuda, rng, T, E, kr, N, K, rac_k)
+    x, w, logits, r, xq, s_w, c_w, sf_w, w_sel, rac_ld = _setup(cuda, rng, T, E, kr, N, K, rac_k, align)
     h = torch.full((r.m_pad_max, I), float("nan"), dtype=torch.bfloat16, device=cuda)
     h_amax = torch.full((1,), 123.0, dtype=torch.float32, device=cuda)
     api.grouped_gemm(xq.codes, xq.scales, xq.s_t, r.m_pad_max, c_w, sf_w, s_w, N, K, E, r.offsets,
-                     rac_ld=rac_ld, rho=xq.r_sel, w_sel=w_sel, epilogue=api.EPI_SWIGLU_BF16,
+                     seg_align=align, rac_ld=rac_ld, rho=xq.r_sel, w_sel=w_sel, epilogue=api.EPI_SWIGLU_BF16,
                      row_token=r.row_token, row_gate=r.row_gate, out=h, amax_out=h_amax)
     y = torch.zeros(T, N, dtype=torch.float32, device=cuda)
     api.grouped_gemm(xq.codes, xq.scales, xq.s_t, r.m_pad_max, c_w, sf_w, s_w, N, K, E, r.offsets,
-                     rac_ld=rac_ld, rho=xq.r_sel, w_sel=w_sel, epilogue=api.EPI_SCATTER_ADD_F32,
+                     seg_align=align, rac_ld=rac_ld, rho=xq.r_sel, w_sel=w_sel, epilogue=api.EPI_SCATTER_ADD_F32,
                      row_token=r.row_token, row_gate=r.row_gate, out=y)
     torch.cuda.synchronize()
     idx, gate, ys = _oracle_rows(x, w, logits, kr, rac_k, xq.sel.cpu().numpy())

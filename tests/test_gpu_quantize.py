@@ -157,20 +157,21 @@ def test_qdq_weights_parity(cuda, G, rows, cols):
         assert np.array_equal(unswizzle(scales[g], rows, cols), ref.sf)
 
 
-@pytest.mark.parametrize("T,E,kr", [(512, 8, 2), (1000, 128, 8), (64, 1, 1), (3, 16, 4), (4096, 256, 8)])
-def test_route_parity(cuda, T, E, kr):
+@pytest.mark.parametrize("T,E,kr,align", [(512, 8, 2, 128), (1000, 128, 8, 128), (64, 1, 1, 128), (3, 16, 4, 128),
+                                          (4096, 256, 8, 128), (1000, 128, 8, 256), (700, 8, 2, 256)])
+def test_route_parity(cuda, T, E, kr, align):
     rng = np.random.default_rng(T + E)
     logits = rng.standard_normal((T, E)).astype(np.float32)
     if E > 4:
         logits[0, [1, 3]] = 5.0      # tie
-    r = api.route(torch.from_numpy(logits).to(cuda), kr)
+    r = api.route(torch.from_numpy(logits).to(cuda), kr, seg_align=align)
     torch.cuda.synchronize()
     idx, gate = oracle.route(logits, kr)
     assert np.array_equal(r.topk_idx.cpu().numpy(), idx)
     np.testing.assert_allclose(r.topk_gate.cpu().numpy(), gate, rtol=2e-6, atol=1e-7)
     off = r.offsets.cpu().numpy()
     counts = np.bincount(idx.reshape(-1), minlength=E)
-    padded = -(-counts // 128) * 128
+    padded = -(-counts // align) * align
     assert np.array_equal(off, np.concatenate([[0], np.cumsum(padded)]))
     dst = r.dst_row.cpu().numpy()
     tok = r.row_token.cpu().numpy()
