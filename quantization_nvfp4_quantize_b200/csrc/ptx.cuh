@@ -96,6 +96,20 @@ __device__ __forceinline__ void bulk_reduce_add_f32(void *dst, uint32_t src, uin
                  ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(src), "r"(bytes) : "memory");
 }
 
+// 16-byte vector add-reduction of four f32 into global memory (relaxed, gpu scope).
+__device__ __forceinline__ void red_add_v4_f32(float *dst, float4 v)
+{
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
+                 ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+}
+
+// 16-byte vector store of four f32.
+__device__ __forceinline__ void st_v4_f32(float *dst, float4 v)
+{
+    asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until this thread's bulk groups have finished reading shared memory.
