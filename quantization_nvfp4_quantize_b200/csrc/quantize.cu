@@ -150,6 +150,15 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
     uint8_t *scales = p.scales ? p.scales + g * p.scales_gstride : nullptr;
     __nv_bfloat16 *qdq = p.qdq ? p.qdq + g * p.qdq_gstride : nullptr;
 
+    // E4M3 code -> (d, 1/d) = (fl(sf * s_t), fl(1 / d)): a block scale takes at
+    // most 127 values per tensor, so each is computed once here rather than
+    // once per block (same arithmetic, same values).
+    __shared__ float2 dtab[128];
+    __shared__ longlong2 fan[QTHREADS / 32][32];                 // per-warp fan-out offsets of one row
+    if (threadIdx.x < 128) {
+        const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), s_t);
+        dtab[threadIdx.x] = make_float2(d, d == 0.0f ? 0.0f : __frcp_rn(d));
+    }
     if (threadIdx.x == 0) {
         for (int st = 0; st < QSTAGES; ++st) {
             ptx::mbar_init(ptx::smem_u32(&full_bar[st]), 1);
@@ -199,7 +208,13 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
 #pragma unroll
             for (int k = 1; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            BlockScale bs = block_scale(m, s_t, r6);
+            BlockScale bs;
+            bs.sf_code = cvt_e4m3(__fmul_rn(m, r6));
+            {
+                const float2 dr = dtab[bs.sf_code];
+                bs.d = dr.x;
+                bs.rcp = dr.y;
+            }
             float xh[8];
             uint32_t cw = quant8(v, bs, xh);
 
@@ -229,16 +244,30 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
                           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[7])) << 16);
                     *reinterpret_cast<uint4 *>(qdq + r * K + c) = o;
                 }
-                if (codes) {
-                    const int nd = p.dst_rows ? p.fanout : 1;
-                    for (int j = 0; j < nd; ++j) {
-                        int64_t dst = p.dst_rows ? (int64_t)p.dst_rows[r * p.fanout + j] : r;
-                        if (dst < 0) continue;
-                        *reinterpret_cast<uint32_t *>(codes + dst * (K >> 1) + (c >> 1)) = cw;
-                        if ((lane & 7) == 0)
-                            *reinterpret_cast<uint32_t *>(scales + sf_offset(dst, kb0, K)) = sw;
-                    }
+                if (codes && !p.dst_rows) {
+                    *reinterpret_cast<uint32_t *>(codes + r * (K >> 1) + (c >> 1)) = cw;
+                    if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(scales + sf_offset(r, kb0, K)) = sw;
                 }
+            }
+            if (codes && p.dst_rows) {
+                // fan-out: lane j < fanout fetches destination j of this row and
+                // stages its code / scale-atom row offsets in shared memory; the
+                // warp then writes the row's codes (128 contiguous bytes) and
+                // scale words to each destination.
+                if (lane < p.fanout) {
+                    const int64_t dst = p.dst_rows[r * p.fanout + lane];
+                    fan[warp][lane] = dst >= 0 ? make_longlong2(dst * (K >> 1), sf_offset(dst, 0, K))
+                                               : make_longlong2(-1, 0);
+                }
+                __syncwarp();
+                const int64_t sf_col_off = (kb0 >> 2) * 512;
+                for (int j = 0; j < p.fanout; ++j) {
+                    const longlong2 o = fan[warp][j];
+                    if (o.x < 0 || !active) continue;
+                    *reinterpret_cast<uint32_t *>(codes + o.x + (c >> 1)) = cw;
+                    if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(scales + o.y + sf_col_off) = sw;
+                }
+                __syncwarp();
             }
         }
         if (SCORE) {
@@ -644,8 +673,8 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
     NVFP4_REQUIRE(aligned16(x_dev) && aligned16(codes_dev) && aligned16(scales_dev),
                   NVFP4_ERR_ALIGNMENT,
                   "nvfp4_quantize: x, codes and scales must be 16-byte aligned");
-    NVFP4_REQUIRE(dst_rows_dev == nullptr || fanout >= 1, NVFP4_ERR_INVALID_ARG,
-                  "nvfp4_quantize: fanout must be >= 1 with dst_rows");
+    NVFP4_REQUIRE(dst_rows_dev == nullptr || (fanout >= 1 && fanout <= 32), NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_quantize: fanout must be in [1, 32] with dst_rows");
     NVFP4_REQUIRE(dst_rows_dev != nullptr || M_out >= M, NVFP4_ERR_INVALID_ARG,
                   "nvfp4_quantize: M_out must be >= M without dst_rows");
     NVFP4_REQUIRE(rac_k >= 0 && rac_k <= 256 && rac_k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
