@@ -156,6 +156,8 @@ def run_ours(args):
     import torch
     from quantization_nvfp4_quantize_b200 import workloads as wl, api
     from quantization_nvfp4_quantize_b200.moe import MoELayerW4A4
+    if wl.CONFIGS[args.workload].w4a16:
+        return run_ours_w4a16(args)
 
     ws, rank = init_dist("nccl" if torch.cuda.is_available() else "gloo")
     _, _, local = dist_env()
@@ -256,6 +258,140 @@ def run_ours(args):
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=8)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return out
+
+
+METRIC_W4A16 = "W4A16 BF16 grouped MoE GEMM TFLOPS and % BF16 peak; weight QDQ GB/s and % HBM"
+QDQ_BYTES_PER_ELEM = 4.0    # 2 B bf16 weight read + 2 B bf16 fake-quantized weight written
+
+
+def run_ours_w4a16(args):
+    """Trainer-side step (asymmetric QAT): NVFP4 fake quantization of every
+    expert weight (they change every optimizer step), then the W4A16 layer
+    forward: routing, routed-row gather of X, BF16 grouped gate/up GEMM with
+    SwiGLU, BF16 grouped down GEMM with router-weighted combine."""
+    import torch
+    from quantization_nvfp4_quantize_b200 import workloads as wl, api
+    from quantization_nvfp4_quantize_b200.moe import MoELayerW4A16
+
+    ws, rank = init_dist("nccl" if torch.cuda.is_available() else "gloo")
+    _, _, local = dist_env()
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = wl.CONFIGS[args.workload]
+    seed = args.seed + rank
+    x = wl.activations(cfg, seed, device=dev)
+    logits = wl.router_logits(cfg, seed, device=dev)
+    w13, w2 = wl.weights(cfg, seed, device=dev)
+    layer = MoELayerW4A16(w13, w2, cfg.tokens, cfg.topk)
+    fl = wl.flops(cfg)
+    step_flops = fl["fp4"]                        # the same two products, in BF16
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.set_weights(w13, w2)
+        return layer.forward(x, logits)
+
+    ev = {"gemm": [], "qdq": []}
+    orig_gemm = api.bf16_grouped_gemm
+    orig_qdq = layer.set_weights
+
+    def timed(kind, fn):
+        def wrap(*a, **k):
+            s_ = torch.cuda.Event(enable_timing=True)
+            e_ = torch.cuda.Event(enable_timing=True)
+            s_.record(stream)
+            out = fn(*a, **k)
+            e_.record(stream)
+            ev[kind].append((s_, e_))
+            return out
+        return wrap
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    api.bf16_grouped_gemm = timed("gemm", orig_gemm)
+    layer.set_weights = timed("qdq", orig_qdq)
+    clocks = ClockSampler(local, enabled=not args.no_clocks)
+    if clocks.proc is not None:
+        time.sleep(0.5)
+    torch.cuda.synchronize()
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    api.bf16_grouped_gemm = orig_gemm
+    layer.set_weights = orig_qdq
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms, dev)
+    gemm_ms = sum(s_.elapsed_time(e_) for s_, e_ in ev["gemm"])
+    qdq_ms = sum(s_.elapsed_time(e_) for s_, e_ in ev["qdq"])
+    p = peaks()
+    bf16_peak = p["bf16_sus"]
+    gemm_tflops = step_flops * args.steps / (gemm_ms * 1e-3) / 1e12
+    w_elems = w13.numel() + w2.numel()
+    qdq_gbs = w_elems * QDQ_BYTES_PER_ELEM * args.steps / (qdq_ms * 1e-3) / 1e9
+
+    # end to end through the public API: X and logits from pinned host memory, Y back
+    xh, lh = x.cpu().pin_memory(), logits.cpu().pin_memory()
+    yh = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
+    xd, ld_ = torch.empty_like(x), torch.empty_like(logits)
+    e_steps = max(1, args.steps // 2)
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        ld_.copy_(lh, non_blocking=True)
+        layer.set_weights(w13, w2)
+        yh.copy_(layer.forward(xd, ld_), non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    s_ = torch.cuda.Event(enable_timing=True)
+    e_ = torch.cuda.Event(enable_timing=True)
+    s_.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e_.record(stream)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(s_.elapsed_time(e_), dev)
+    out = {
+        "metric": METRIC_W4A16,
+        "value": round(step_flops * args.steps * ws / (ms_max * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 (fp32 accum), NVFP4 fake-quantized weights", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: T={cfg.tokens} H={cfg.hidden} I={cfg.inter} E={cfg.experts} "
+                               f"top-{cfg.topk}, weight QDQ every step",
+                   "l2": "inputs larger than L2 (bf16 weights 1.2 GB)", "parallelism": f"replicas x{ws}"},
+        "roofline": {"bound": "tensor", "kernel": "k_moe_gemm (BF16 stages)",
+                     "achieved": round(gemm_tflops, 1), "peak": round(bf16_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_tflops / bf16_peak, 4), "traffic": None,
+                     "peak_source": f"{p['source']} bf16 sustained",
+                     "gemm_ms_per_step": round(gemm_ms / args.steps, 4), "launches_per_step": 2},
+        "qdq": {"gbs": round(qdq_gbs, 1), "peak_gbs": p["hbm"], "frac": round(qdq_gbs / p["hbm"], 4),
+                "ms_per_step": round(qdq_ms / args.steps, 4), "bytes_per_elem": QDQ_BYTES_PER_ELEM,
+                "elems_per_step": w_elems},
+        "e2e": {"value": round(step_flops * e_steps * ws / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": xh.numel() * xh.element_size() + lh.numel() * lh.element_size(),
+                "d2h_bytes_per_step": yh.numel() * yh.element_size()},
+        # per step: 2 x (amax + quantize) for the weights, route (2), gather, 2 GEMMs
+        "gpu_launches": 9 * args.steps,
+        "clocks": clk,
+    }
     if rank == 0:
         print(json.dumps(out), flush=True)
     return out

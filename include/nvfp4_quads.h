@@ -325,6 +325,40 @@ NVFP4_API nvfp4_status moe_w4a4_grouped_gemm_rac(
     int32_t *dev_status, void *stream);
 
 /* --------------------------------------------------------------------------
+ * moe_bf16_grouped_gemm -- the trainer-side W4A16 expert GEMM
+ * (gist.science/it 2.2 A: the trainer fake-quantizes the weights to NVFP4
+ * and keeps activations in BF16): BF16 A x BF16 B on the tensor cores
+ * (kind::f16, f32 accumulation in TMEM), B normally the nvfp4_qdq_weights
+ * output.  For every routed row r of expert e and output feature n:
+ *   y[r,n] = sum_k a[r,k] b_e[n,k]
+ * with the same three epilogues as moe_w4a4_grouped_gemm_rac (unit tensor
+ * scales).
+ *   a_dev     bf16 [M_pad_max x lda], rows in routed order (e.g. from
+ *             moe_gather_rows_bf16, or the SwiGLU output of the first GEMM).
+ *   b_dev     bf16 [E x N x K], contiguous.
+ *   offsets_dev, seg_align, epilogue, row_token_dev, row_gate_dev, out_dev,
+ *   ld_out, amax_out_dev: as for moe_w4a4_grouped_gemm_rac.
+ * Shapes: K % 64 == 0, N % 256 == 0 (SWIGLU: I % 128 == 0), lda >= K and
+ * lda % 8 == 0, M_pad_max a multiple of seg_align, E <= 256.  Pointers 16-byte
+ * aligned.  Errors as for moe_w4a4_grouped_gemm_rac.
+ *
+ * moe_gather_rows_bf16 -- the W4A16 path's activation fan-out: token row t of
+ * x (bf16 [T x ldx]) is copied to rows dst_rows[t*fanout + j] (j < fanout,
+ * 1 <= fanout <= 32, negative entries skipped) of out (bf16 [M_out x ld_out]);
+ * other rows of out are not touched.  K % 8 == 0, ldx and ld_out >= K and
+ * multiples of 8, pointers 16-byte aligned.
+ * -------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status moe_bf16_grouped_gemm(
+    const void *a_dev, int64_t lda, int64_t M_pad_max, const void *b_dev, int64_t N, int64_t K, int32_t E,
+    const int32_t *offsets_dev, int32_t seg_align, int32_t epilogue, const int32_t *row_token_dev,
+    const float *row_gate_dev, void *out_dev, int64_t ld_out, float *amax_out_dev, int32_t *dev_status,
+    void *stream);
+
+NVFP4_API nvfp4_status moe_gather_rows_bf16(const void *x_dev, int64_t T, int64_t K, int64_t ldx,
+                                            const int32_t *dst_rows_dev, int32_t fanout, void *out_dev,
+                                            int64_t ld_out, int64_t M_out, void *stream);
+
+/* --------------------------------------------------------------------------
  * nvfp4_debug_encode -- runs the library's element and scale encoders on n
  * arbitrary floats (for validation against an independent definition):
  *   e2m1_dev[i] = E2M1 code of in[i] (nearest even, saturating, sign bit

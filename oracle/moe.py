@@ -79,10 +79,48 @@ def layer(x, logits, w13q, w2q, kr, k_x, k_h):
     return out
 
 
+def layer_w4a16(x, logits, w13, w2, kr, experts=None):
+    """Trainer-side W4A16 layer (gist.science/it 2.2 A: NVFP4 fake-quantized
+    weights, BF16 activations):
+
+        Wq       = bf16(QDQ(W_e)) per expert tensor (oracle.qdq)
+        y13[t,j] = X[t] Wq13_e^T              binary64 of the bf16 values
+        h[t,j]   = bf16(silu(y13[:, :I]) * y13[:, I:])
+        y2[t,j]  = h[t,j] Wq2_e^T
+        Y[t]     = sum_j g[t,j] y2[t,j]
+
+    ``experts``: optional dict e -> (Wq13_e, Wq2_e) bf16 bits, to reuse the
+    weight fake-quantization between calls; missing experts are quantized
+    here.  Returns dict(Y, h64, h_bf16, idx, gate)."""
+    from . import qdq
+    idx, gate = route(logits, kr)
+    T = x.shape[0]
+    inter = w13.shape[1] // 2
+    H = w2.shape[1]
+    cache = {} if experts is None else experts
+    xf = bf16_to_f32(x).astype(np.float64)
+    rows_t = np.repeat(np.arange(T), kr)
+    flat = idx.reshape(-1)
+    h = np.zeros((T * kr, inter), np.float64)
+    for e in np.unique(flat):
+        if e not in cache:
+            cache[e] = (qdq(w13[e])[0], qdq(w2[e])[0])
+        rows = np.nonzero(flat == e)[0]
+        h[rows] = swiglu(xf[rows_t[rows]] @ bf16_to_f32(cache[e][0]).astype(np.float64).T, inter)
+    hb = f32_to_bf16(h.astype(np.float32))
+    hf = bf16_to_f32(hb).astype(np.float64)
+    y2 = np.zeros((T * kr, H), np.float64)
+    for e in np.unique(flat):
+        rows = np.nonzero(flat == e)[0]
+        y2[rows] = hf[rows] @ bf16_to_f32(cache[e][1]).astype(np.float64).T
+    Y = (y2.reshape(T, kr, H) * gate[:, :, None]).sum(axis=1)
+    return dict(Y=Y, h64=h, h_bf16=hb, idx=idx, gate=gate)
+
+
 def tokens_sample(x, logits, tokens):
     """Restrict a layer's token inputs to a subset of tokens (used for the
     large workloads, where the oracle runs on a sample)."""
     return x[tokens], logits[tokens]
 
 
-__all__ = ["quantize_weights", "gate_up", "down", "layer", "tokens_sample", "bf16_to_f32"]
+__all__ = ["quantize_weights", "gate_up", "down", "layer", "layer_w4a16", "tokens_sample", "bf16_to_f32"]

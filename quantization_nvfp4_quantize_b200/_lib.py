@@ -45,6 +45,11 @@ SIGNATURES = {
                                             c_void_p, c_int64, c_int64, c_int32, c_void_p, c_int32, c_int32, c_void_p,
                                             c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_void_p,
                                             c_void_p, c_void_p]),
+    "moe_bf16_grouped_gemm": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_int64, c_int32, c_void_p,
+                                        c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
+                                        c_void_p]),
+    "moe_gather_rows_bf16": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int32, c_void_p, c_int64,
+                                       c_int64, c_void_p]),
     "nvfp4_debug_encode": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
 }
 

@@ -184,6 +184,33 @@ def grouped_gemm(a_codes, a_scales, a_s_t, m_pad_max, b_codes, b_scales, b_s_t, 
     return out
 
 
+def bf16_grouped_gemm(a, m_pad_max, b, N, K, E, offsets, *, seg_align=128, epilogue=EPI_STORE_F32,
+                      row_token=None, row_gate=None, out=None, ld_out=None, amax_out=None, dev_status=None):
+    """moe_bf16_grouped_gemm (see the header): bf16 A [m_pad_max x lda] in
+    routed order times bf16 B [E x N x K]."""
+    lib = _lib.load()
+    assert a.dtype == BF16 and b.dtype == BF16 and b.is_contiguous()
+    if ld_out is None:
+        ld_out = out.stride(0)
+    check(lib.moe_bf16_grouped_gemm(_p(a), a.stride(0), m_pad_max, _p(b), N, K, E, _p(offsets), seg_align, epilogue,
+                                    _p(row_token), _p(row_gate), _p(out), ld_out, _p(amax_out), _p(dev_status),
+                                    _stream(out.device)))
+    return out
+
+
+def gather_rows_bf16(x: torch.Tensor, dst_rows: torch.Tensor, m_out: int, *, out=None):
+    """moe_gather_rows_bf16: token rows of x to their routed rows (dst_rows
+    int32 [T x fanout]); rows of `out` not named are left as they are."""
+    lib = _lib.load()
+    assert x.dtype == BF16 and x.dim() == 2 and dst_rows.dtype == I32
+    T, K = x.shape
+    if out is None:
+        out = torch.zeros(m_out, K, dtype=BF16, device=x.device)
+    check(lib.moe_gather_rows_bf16(_p(x), T, K, x.stride(0), _p(dst_rows), dst_rows.shape[1], _p(out), out.stride(0),
+                                   m_out, _stream(x.device)))
+    return out
+
+
 def debug_encode(v: torch.Tensor):
     """nvfp4_debug_encode: (E2M1 codes, E4M3 codes) of float32 values."""
     lib = _lib.load()

@@ -381,7 +381,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                     issued_any = true;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (ok && nrk > 0) {
+                if (ok && nrk > 0 && nkb > 0) {
                     // the BF16 MMAs accumulate into the same TMEM tile: wait for
                     // the FP4 MMAs to complete first
                     if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->drain), 1);
@@ -389,6 +389,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                     if (!wait_bar(ptx::smem_u32(&sh->drain), drain_phase, abort_flag, p.dev_status)) { ok = false; }
                     drain_phase ^= 1u;
                     ptx::tc_fence_after();
+                }
+                if (ok && nrk > 0) {
                     for (int rk = 0; rk < nrk && ok; ++rk) {
                         if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status) ||
                             !wait_bar(ptx::smem_u32(&sh->sf_full[stage]), phase, abort_flag, p.dev_status)) {
@@ -402,8 +404,10 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                         for (int kk = 0; kk < 4; ++kk) {
                             uint64_t ad = ptx::make_sdesc(sa + 32 * kk, 16, 1024, 2);
                             uint64_t bd = ptx::make_sdesc(sb + 32 * kk, 16, 1024, 2);
-                            if (PAIR) ptx::mma_bf16_pair(tmem + ACC_COL, ad, bd, idesc16, 1u);
-                            else ptx::mma_bf16(tmem + ACC_COL, ad, bd, idesc16, 1u);
+                            // without an FP4 part (BF16-only GEMM) the tile's first MMA overwrites
+                            const uint32_t acc = (nkb > 0 || rk > 0 || kk > 0) ? 1u : 0u;
+                            if (PAIR) ptx::mma_bf16_pair(tmem + ACC_COL, ad, bd, idesc16, acc);
+                            else ptx::mma_bf16(tmem + ACC_COL, ad, bd, idesc16, acc);
                         }
                         if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->empty[stage]), 3);
                         else ptx::tc_commit(ptx::smem_u32(&sh->empty[stage]));
@@ -480,7 +484,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
         const int q = warp & 3;
         const int half = (warp - EPI_WARP0) >> 2;
         const int row_in_tile = (int)rank * 128 + q * 32 + lane;
-        const float s_a = *p.a_s_t;
+        const float s_a = p.a_s_t ? *p.a_s_t : 1.0f;       // null: unit tensor scales (BF16 GEMM)
         const uint32_t empty_bar = PAIR ? ptx::mapa_shared(ptx::smem_u32(&sh->tmem_empty), 0)
                                         : ptx::smem_u32(&sh->tmem_empty);
         int iter = 0;
@@ -515,7 +519,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                 else ptx::mbar_arrive(empty_bar);
             }
 
-            const float scale = __fmul_rn(s_a, p.b_s_t[e]);
+            const float scale = __fmul_rn(s_a, p.b_s_t ? p.b_s_t[e] : 1.0f);
             const int64_t r = (int64_t)m0 + row_in_tile;
             const int token = p.row_token[r];
             if (p.epilogue == MOE_EPI_SWIGLU_BF16) {
@@ -632,6 +636,42 @@ static nvfp4_status launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, con
     return check_launch("k_moe_gemm");
 }
 
+
+// Tile order and launch shape (1-SM or 2-SM tiles, stages), then launch.
+static nvfp4_status dispatch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, const CUtensorMap &tm_ra,
+                             const CUtensorMap &tm_rb, const CUtensorMap &tm_sfa, const CUtensorMap &tm_sfb,
+                             Params &p, int64_t M_pad_max, int seg_align, cudaStream_t st)
+{
+    const int epilogue = p.epilogue;
+    const bool pair = seg_align == 256;
+    const int64_t n_tiles = epilogue == MOE_EPI_SWIGLU_BF16 ? p.inter / 128 : p.N / BN;
+    // Tile order: the scatter-add epilogue reduces into token rows that every
+    // expert touches; grouping 2 n-tiles (512 output columns) keeps the band
+    // of output being reduced into small enough to stay in L2 while all
+    // experts' contributions to it arrive (16384 tokens x 4096 f32: 1114 us
+    // in plain order, 937 us in groups of 2).  NVFP4_GEMM_NGROUP overrides
+    // (must divide the n-tile count).
+    int n_group = (int)n_tiles;
+    if (epilogue == MOE_EPI_SCATTER_ADD_F32 && n_tiles % 2 == 0) n_group = 2;
+    if (const char *env = getenv("NVFP4_GEMM_NGROUP")) {
+        const int g = atoi(env);
+        if (g > 0 && n_tiles % g == 0) n_group = g;
+    }
+    p.n_group = n_group;
+    const int64_t max_tiles = (M_pad_max / seg_align) * n_tiles;
+    const bool swiglu = epilogue == MOE_EPI_SWIGLU_BF16;
+    if (pair) {
+        // 5 stages; the f32 epilogues add their transpose tiles
+        const int units = (int)std::min<int64_t>(num_sms() / 2, max_tiles);
+        return swiglu ? launch<5, true, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
+                      : launch<5, true, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
+    }
+    // SwiGLU (bf16 out): 4 stages; f32 epilogues: 3 stages + transpose tiles
+    const int units = (int)std::min<int64_t>(num_sms(), max_tiles);
+    return swiglu ? launch<4, false, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
+                  : launch<3, false, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
+}
+
 }  // namespace gemm
 }  // namespace nvfp4
 
@@ -730,30 +770,70 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
     p.dev_status = dev_status;
     if (p.amax_out && cudaMemsetAsync(p.amax_out, 0, sizeof(float), st) != cudaSuccess)
         return check_launch("moe_w4a4_grouped_gemm_rac: memset");
-    const int64_t n_tiles = epilogue == MOE_EPI_SWIGLU_BF16 ? inter / 128 : N / BN;
-    // Tile order: the scatter-add epilogue reduces into token rows that every
-    // expert touches; grouping 2 n-tiles (512 output columns) keeps the band
-    // of output being reduced into small enough to stay in L2 while all
-    // experts' contributions to it arrive (16384 tokens x 4096 f32: 1114 us
-    // in plain order, 937 us in groups of 2).  NVFP4_GEMM_NGROUP overrides
-    // (must divide the n-tile count).
-    int n_group = (int)n_tiles;
-    if (epilogue == MOE_EPI_SCATTER_ADD_F32 && n_tiles % 2 == 0) n_group = 2;
-    if (const char *env = getenv("NVFP4_GEMM_NGROUP")) {
-        const int g = atoi(env);
-        if (g > 0 && n_tiles % g == 0) n_group = g;
+    return dispatch(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, M_pad_max, seg_align, st);
+}
+
+extern "C" nvfp4_status moe_bf16_grouped_gemm(
+    const void *a_dev, int64_t lda, int64_t M_pad_max, const void *b_dev, int64_t N, int64_t K, int32_t E,
+    const int32_t *offsets_dev, int32_t seg_align, int32_t epilogue, const int32_t *row_token_dev,
+    const float *row_gate_dev, void *out_dev, int64_t ld_out, float *amax_out_dev, int32_t *dev_status, void *stream)
+{
+    using namespace nvfp4::gemm;
+    cudaStream_t st = (cudaStream_t)stream;
+    NVFP4_REQUIRE(a_dev && b_dev && offsets_dev && row_token_dev && out_dev, NVFP4_ERR_INVALID_ARG,
+                  "moe_bf16_grouped_gemm: null pointer");
+    NVFP4_REQUIRE(epilogue >= 0 && epilogue <= 2, NVFP4_ERR_INVALID_ARG, "moe_bf16_grouped_gemm: bad epilogue");
+    NVFP4_REQUIRE(seg_align == 128 || seg_align == 256, NVFP4_ERR_INVALID_ARG,
+                  "moe_bf16_grouped_gemm: seg_align must be 128 or 256");
+    NVFP4_REQUIRE(epilogue != MOE_EPI_SCATTER_ADD_F32 || row_gate_dev, NVFP4_ERR_INVALID_ARG,
+                  "moe_bf16_grouped_gemm: scatter-add needs row_gate");
+    NVFP4_REQUIRE(E >= 1 && E <= MAX_E, NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_bf16_grouped_gemm: 1 <= E <= 256");
+    NVFP4_REQUIRE(K >= 64 && K % 64 == 0 && K < (1 << 20), NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "moe_bf16_grouped_gemm: K must be a positive multiple of 64 (K=%lld)", (long long)K);
+    NVFP4_REQUIRE(N >= 256 && N % 256 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "moe_bf16_grouped_gemm: N must be a positive multiple of 256 (N=%lld)", (long long)N);
+    NVFP4_REQUIRE(lda >= K && lda % 8 == 0, NVFP4_ERR_ALIGNMENT,
+                  "moe_bf16_grouped_gemm: lda must be >= K and a multiple of 8");
+    NVFP4_REQUIRE(M_pad_max >= seg_align && M_pad_max % seg_align == 0 && M_pad_max < (1ll << 31),
+                  NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_bf16_grouped_gemm: M_pad_max must be a positive multiple of seg_align");
+    NVFP4_REQUIRE((int64_t)E * N < (1ll << 31), NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_bf16_grouped_gemm: E*N too large");
+    const int inter = (int)(N / 2);
+    if (epilogue == MOE_EPI_SWIGLU_BF16) {
+        NVFP4_REQUIRE(inter % 128 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_bf16_grouped_gemm: SwiGLU needs I % 128 == 0");
+        NVFP4_REQUIRE(ld_out >= inter && ld_out % 8 == 0, NVFP4_ERR_ALIGNMENT,
+                      "moe_bf16_grouped_gemm: SwiGLU ld_out must be >= N/2 and a multiple of 8");
+    } else {
+        NVFP4_REQUIRE(ld_out >= N && ld_out % 4 == 0, NVFP4_ERR_ALIGNMENT,
+                      "moe_bf16_grouped_gemm: ld_out must be >= N and a multiple of 4");
     }
-    p.n_group = n_group;
-    const int64_t max_tiles = (M_pad_max / seg_align) * n_tiles;
-    const bool swiglu = epilogue == MOE_EPI_SWIGLU_BF16;
-    if (pair) {
-        // SwiGLU (bf16 out): 5 stages; f32 epilogues: 4 stages + staging
-        const int units = (int)std::min<int64_t>(num_sms() / 2, max_tiles);
-        return swiglu ? launch<5, true, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
-                      : launch<5, true, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
-    }
-    // SwiGLU (bf16 out): 4 stages; f32 epilogues: 3 stages + staging
-    const int units = (int)std::min<int64_t>(num_sms(), max_tiles);
-    return swiglu ? launch<4, false, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
-                  : launch<3, false, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
+    NVFP4_REQUIRE(aligned16(a_dev) && aligned16(b_dev) && aligned16(out_dev), NVFP4_ERR_ALIGNMENT,
+                  "moe_bf16_grouped_gemm: pointers must be 16-byte aligned");
+
+    // A and B travel the kernel's BF16 (kind::f16) stages, K / 64 of them per
+    // tile, with no FP4 stage and unit tensor scales.
+    CUtensorMap tm_ra, tm_rb;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    const bool ok = make_tmap_2d(&tm_ra, a_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)K, (uint64_t)M_pad_max,
+                                 (uint64_t)lda * 2, 64, 128, sw) &&
+                    make_tmap_2d(&tm_rb, b_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)K, (uint64_t)E * N,
+                                 (uint64_t)K * 2, 64, 128, sw);
+    NVFP4_REQUIRE(ok, NVFP4_ERR_CUDA, "moe_bf16_grouped_gemm: tensor map encoding failed");
+
+    Params p{};
+    p.N = N;
+    p.K = 0;                          // no FP4 stages
+    p.E = E;
+    p.offsets = offsets_dev;
+    p.rac_ld = (int)K;                // the BF16 stages cover all of K
+    p.epilogue = epilogue;
+    p.inter = inter;
+    p.row_token = row_token_dev;
+    p.row_gate = row_gate_dev;
+    p.out = out_dev;
+    p.ld_out = ld_out;
+    p.amax_out = (epilogue == MOE_EPI_SWIGLU_BF16) ? reinterpret_cast<unsigned int *>(amax_out_dev) : nullptr;
+    p.dev_status = dev_status;
+    if (p.amax_out && cudaMemsetAsync(p.amax_out, 0, sizeof(float), st) != cudaSuccess)
+        return check_launch("moe_bf16_grouped_gemm: memset");
+    return dispatch(tm_ra, tm_rb, tm_ra, tm_rb, tm_ra, tm_rb, p, M_pad_max, seg_align, st);
 }

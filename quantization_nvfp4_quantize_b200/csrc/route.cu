@@ -140,9 +140,45 @@ __global__ void __launch_bounds__(1024) k_route_assign(const int32_t *__restrict
     }
 }
 
+// One CTA per (token row, 2048-column chunk): each thread loads 8 bf16 of the
+// row once and stores them to every destination row.
+__global__ void __launch_bounds__(256) k_gather_rows_bf16(const uint4 *__restrict__ x, int64_t K, int64_t ldx,
+                                                          const int32_t *__restrict__ dst_rows, int fanout,
+                                                          uint4 *__restrict__ out, int64_t ld_out, int64_t M_out)
+{
+    const int64_t t = blockIdx.x;
+    const int64_t col = ((int64_t)blockIdx.y * 256 + threadIdx.x) * 8;
+    if (col >= K) return;
+    const uint4 v = x[(t * ldx + col) >> 3];
+    for (int j = 0; j < fanout; ++j) {
+        const int64_t d = dst_rows[t * fanout + j];
+        if (d >= 0 && d < M_out) out[(d * ld_out + col) >> 3] = v;
+    }
+}
+
 }  // namespace nvfp4
 
 using namespace nvfp4;
+
+extern "C" nvfp4_status moe_gather_rows_bf16(const void *x_dev, int64_t T, int64_t K, int64_t ldx,
+                                             const int32_t *dst_rows_dev, int32_t fanout, void *out_dev,
+                                             int64_t ld_out, int64_t M_out, void *stream)
+{
+    NVFP4_REQUIRE(T >= 0 && K >= 0 && M_out >= 0, NVFP4_ERR_INVALID_ARG, "moe_gather_rows_bf16: negative size");
+    if (T == 0 || K == 0) return NVFP4_OK;
+    NVFP4_REQUIRE(x_dev && dst_rows_dev && out_dev, NVFP4_ERR_INVALID_ARG, "moe_gather_rows_bf16: null pointer");
+    NVFP4_REQUIRE(fanout >= 1 && fanout <= 32, NVFP4_ERR_INVALID_ARG, "moe_gather_rows_bf16: fanout must be in [1, 32]");
+    NVFP4_REQUIRE(K % 8 == 0 && ldx >= K && ldx % 8 == 0 && ld_out >= K && ld_out % 8 == 0, NVFP4_ERR_ALIGNMENT,
+                  "moe_gather_rows_bf16: K, ldx and ld_out must be multiples of 8 with ldx, ld_out >= K");
+    NVFP4_REQUIRE(aligned16(x_dev) && aligned16(out_dev), NVFP4_ERR_ALIGNMENT,
+                  "moe_gather_rows_bf16: pointers must be 16-byte aligned");
+    NVFP4_REQUIRE(T < (1ll << 31), NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_gather_rows_bf16: too many rows");
+    dim3 grid((unsigned)T, (unsigned)((K + 2047) / 2048));
+    k_gather_rows_bf16<<<grid, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const uint4 *>(x_dev), K, ldx,
+                                                               dst_rows_dev, fanout, reinterpret_cast<uint4 *>(out_dev),
+                                                               ld_out, M_out);
+    return check_launch("k_gather_rows_bf16");
+}
 
 extern "C" size_t moe_route_workspace_size(int64_t T, int32_t E)
 {

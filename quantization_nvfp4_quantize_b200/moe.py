@@ -108,6 +108,67 @@ class MoELayerW4A4:
         return r
 
 
+class MoELayerW4A16:
+    """Trainer-side asymmetric QAT layer (gist.science/it 2.2 A): the expert
+    weights are fake-quantized to NVFP4 (nvfp4_qdq_weights: bf16 ->
+    NVFP4 with each expert tensor's own scale -> bf16), activations stay
+    BF16, and both expert GEMMs run as BF16 grouped GEMMs on the tensor cores:
+
+      1. moe_route               as in MoELayerW4A4
+      2. moe_gather_rows_bf16    X rows to their routed rows
+      3. BF16 grouped GEMM       X Wq13^T, epilogue SwiGLU -> h bf16
+      4. BF16 grouped GEMM       h Wq2^T, epilogue router-weighted scatter-add
+                                 into Y [T x H] fp32
+    """
+
+    def __init__(self, w13: torch.Tensor, w2: torch.Tensor, tokens: int, topk: int, seg_align: int = 256):
+        assert w13.dtype == torch.bfloat16 and w2.dtype == torch.bfloat16
+        E, N13, H = w13.shape
+        E2, H2, I = w2.shape
+        assert E2 == E and H2 == H and N13 == 2 * I
+        dev = w13.device
+        self.E, self.H, self.I, self.T, self.k_r = E, H, I, tokens, topk
+        self.wq13 = torch.empty_like(w13)
+        self.wq2 = torch.empty_like(w2)
+        self.s13 = torch.empty(E, dtype=torch.float32, device=dev)
+        self.s2 = torch.empty(E, dtype=torch.float32, device=dev)
+        lib = api._lib.load()
+        self.ws_qdq = api._ws(max(lib.nvfp4_qdq_workspace_size(E, 2 * I, H), lib.nvfp4_qdq_workspace_size(E, H, I)), dev)
+        self.set_weights(w13, w2)
+        self.seg_align = seg_align
+        self.m_pad = api.padded_rows_bound(tokens, topk, E, seg_align)
+        self.xr = torch.zeros(self.m_pad, H, dtype=torch.bfloat16, device=dev)
+        self.h = torch.empty(self.m_pad, I, dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty(tokens, H, dtype=torch.float32, device=dev)
+        self.routing = None
+
+    def set_weights(self, w13: torch.Tensor, w2: torch.Tensor):
+        """Fake-quantize new bf16 weights into the layer (the per-step work of
+        QAT, where the weights change every optimizer step)."""
+        lib = api._lib.load()
+        st = api._stream(w13.device)
+        for w, wq, s_t in ((w13, self.wq13, self.s13), (w2, self.wq2, self.s2)):
+            assert w.shape == wq.shape and w.dtype == torch.bfloat16 and w.is_contiguous()
+            G, rows, cols = w.shape
+            api.check(lib.nvfp4_qdq_weights(api._p(w), G, rows, cols, api._p(wq), api._p(s_t), None, None,
+                                            api._p(self.ws_qdq), self.ws_qdq.numel(), st))
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor) -> torch.Tensor:
+        E, H, I = self.E, self.H, self.I
+        r = api.route(logits, self.k_r, self.m_pad, self.seg_align) if self.routing is None else self._route_into(logits)
+        self.routing = r
+        api.gather_rows_bf16(x, r.dst_row, self.m_pad, out=self.xr)
+        api.bf16_grouped_gemm(self.xr, self.m_pad, self.wq13, 2 * I, H, E, r.offsets, seg_align=self.seg_align,
+                              epilogue=api.EPI_SWIGLU_BF16, row_token=r.row_token, row_gate=r.row_gate, out=self.h)
+        self.y.zero_()
+        api.bf16_grouped_gemm(self.h, self.m_pad, self.wq2, H, I, E, r.offsets, seg_align=self.seg_align,
+                              epilogue=api.EPI_SCATTER_ADD_F32, row_token=r.row_token, row_gate=r.row_gate,
+                              out=self.y)
+        return self.y
+
+    _route_into = MoELayerW4A4._route_into
+
+
 class DenseLayerW4A4:
     """Single dense W4A4 + RAC layer: Y = Xq Wq^T + RAC, fp32 out (one expert,
     identity routing)."""

@@ -83,6 +83,19 @@ def test_argument_errors_are_synchronous():
     pair_rows = list(args)
     pair_rows[11] = 256                      # M_pad_max (128) is not a multiple of 256
     assert lib.moe_w4a4_grouped_gemm_rac(*pair_rows) == 3
+    # BF16 grouped GEMM (W4A16) and the bf16 row gather
+    bargs = [fake, 256, 128, fake, 256, 256, 1, fake, 128, 0, fake, None, fake, 256, None, None, None]
+    bad = list(bargs)
+    bad[5] = 96                              # K not a multiple of 64
+    assert lib.moe_bf16_grouped_gemm(*bad) == 3
+    bad = list(bargs)
+    bad[1] = 100                             # lda not a multiple of 8
+    assert lib.moe_bf16_grouped_gemm(*bad) == 2
+    bad = list(bargs)
+    bad[9] = 2                               # scatter-add without row_gate
+    assert lib.moe_bf16_grouped_gemm(*bad) == 1
+    assert lib.moe_gather_rows_bf16(fake, 4, 64, 64, fake, 0, fake, 64, 16, None) == 1
+    assert lib.moe_gather_rows_bf16(fake, 4, 60, 64, fake, 2, fake, 64, 16, None) == 2
     # routing
     assert lib.moe_route(fake, 16, 300, 2, fake, fake, 128, fake, fake, fake, fake, 1 << 20, fake, 4096, None) == 3
     assert lib.moe_route(fake, 16, 8, 2, fake, fake, 128, fake, fake, fake, fake, 128, fake, 4096, None) == 1

@@ -114,3 +114,84 @@ def test_moe_token_permutation_permutes_rows():
     perm = rng.permutation(x.shape[0])
     out_p = omoe.layer(x[perm], logits[perm], w13q, w2q, kr=2, k_x=8, k_h=4)
     np.testing.assert_allclose(out_p["Y"], out["Y"][perm], rtol=1e-9, atol=1e-12)
+
+
+# ------------------------------------------------------------------ W4A16 layer
+# Pins of oracle.moe.layer_w4a16 (gist.science/it 2.2 A: NVFP4 fake-quantized
+# weights, BF16 activations) by invariances and by a special case in which the
+# fake quantization is the identity.
+
+def _w4a16_inputs(rng, T=6, H=32, I=16, E=3):
+    x = bf16(rng.standard_normal((T, H)))
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    w13 = bf16(rng.standard_normal((E, 2 * I, H)) * 0.1)
+    w2 = bf16(rng.standard_normal((E, H, I)) * 0.1)
+    return x, logits, w13, w2
+
+
+def test_w4a16_expert_permutation_invariance():
+    rng = np.random.default_rng(21)
+    x, logits, w13, w2 = _w4a16_inputs(rng)
+    perm = np.array([2, 0, 1])
+    a = omoe.layer_w4a16(x, logits, w13, w2, 2)["Y"]
+    b = omoe.layer_w4a16(x, logits[:, perm], w13[perm], w2[perm], 2)["Y"]
+    np.testing.assert_allclose(a, b, rtol=0, atol=0)
+
+
+def test_w4a16_token_permutation_equivariance():
+    rng = np.random.default_rng(22)
+    x, logits, w13, w2 = _w4a16_inputs(rng)
+    perm = rng.permutation(x.shape[0])
+    a = omoe.layer_w4a16(x, logits, w13, w2, 2)["Y"]
+    b = omoe.layer_w4a16(x[perm], logits[perm], w13, w2, 2)["Y"]
+    np.testing.assert_allclose(a[perm], b, rtol=0, atol=0)
+
+
+def test_w4a16_down_weight_scaling_is_exact():
+    # doubling W2 doubles its tensor scale and leaves its codes and block
+    # scales unchanged, so the fake-quantized weight and Y double exactly
+    rng = np.random.default_rng(23)
+    x, logits, w13, w2 = _w4a16_inputs(rng)
+    a = omoe.layer_w4a16(x, logits, w13, w2, 2)["Y"]
+    w2x2 = bf16(oracle.bf16_to_f32(w2) * 2.0)
+    b = omoe.layer_w4a16(x, logits, w13, w2x2, 2)["Y"]
+    np.testing.assert_array_equal(b, 2.0 * a)
+
+
+def test_w4a16_on_grid_weights_reduce_to_dense_ffn():
+    # weights whose every 16-block holds +-6 and E2M1 values with the tensor
+    # max 6 * 448 * 2^-12: every block scale is exactly 448 * 2^-12 / s_t
+    # representable, so fake quantization returns the weights unchanged and
+    # one expert with top-1 routing is the plain SwiGLU FFN
+    rng = np.random.default_rng(24)
+    T, H, I = 5, 32, 16
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
+
+    def on_grid(shape):
+        v = rng.choice(grid, size=shape) * rng.choice([-1, 1], size=shape)
+        v = v.reshape(-1, 16)
+        v[:, 0] = 6.0                          # every block's max is 6
+        return bf16((v.reshape(shape) * 448.0 * 2.0 ** -12).astype(np.float32))
+
+    w13 = on_grid((1, 2 * I, H))
+    w2 = on_grid((1, H, I))
+    assert np.array_equal(oracle.qdq(w13[0])[0], w13[0]) and np.array_equal(oracle.qdq(w2[0])[0], w2[0])
+    x = bf16(rng.standard_normal((T, H)))
+    logits = np.zeros((T, 1), np.float32)
+    out = omoe.layer_w4a16(x, logits, w13, w2, 1)
+    xf = oracle.bf16_to_f32(x).astype(np.float64)
+    g = np.einsum("th,nh->tn", xf, oracle.bf16_to_f32(w13[0]).astype(np.float64))
+    h = g[:, :I] / (1.0 + np.exp(-g[:, :I])) * g[:, I:]
+    hb = oracle.bf16_to_f32(bf16(h.astype(np.float32))).astype(np.float64)
+    y = np.einsum("ti,hi->th", hb, oracle.bf16_to_f32(w2[0]).astype(np.float64))
+    np.testing.assert_allclose(out["Y"], y, rtol=1e-12, atol=0)
+
+
+def test_w4a16_router_weights_sum_over_identical_experts():
+    # two identical experts, top-2: Y = (g0 + g1) y = y, the one-expert layer
+    rng = np.random.default_rng(25)
+    x, logits, w13, w2 = _w4a16_inputs(rng, E=1)
+    one = omoe.layer_w4a16(x, np.zeros((x.shape[0], 1), np.float32), w13, w2, 1)["Y"]
+    two = omoe.layer_w4a16(x, rng.standard_normal((x.shape[0], 2)).astype(np.float32),
+                           np.concatenate([w13, w13]), np.concatenate([w2, w2]), 2)["Y"]
+    np.testing.assert_allclose(two, one, rtol=1e-13, atol=1e-15)
