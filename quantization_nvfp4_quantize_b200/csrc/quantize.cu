@@ -547,50 +547,69 @@ __global__ void k_weights_channel_major(const uint8_t *__restrict__ codes, const
 // (64 bytes) are read as contiguous runs, dequantized (e2m1 * sf, exact in
 // bf16) into a shared [channel][feature] tile, then written out transposed as
 // [feature][ld] rows.
-constexpr int GCM_N = 64;
-constexpr int GCM_TS = GCM_N + 4;                     // padded row of the shared tile (floats)
+constexpr int GCM_N = 128;                           // output features per CTA
 
 __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__restrict__ codes_cm,
                                                               const uint8_t *__restrict__ scales_cm, int64_t N,
                                                               int64_t K, const int32_t *__restrict__ sel, int k,
                                                               int ld, __nv_bfloat16 *__restrict__ out)
 {
-    extern __shared__ float gtile[];                   // [ld][GCM_TS]
+    extern __shared__ float gtile[];                   // [GCM_N features][ld channels]
+    __shared__ float e4[128];                          // E4M3 code -> value (weight scales are non-negative)
+    __shared__ int32_t ssel[256];
     const int64_t e = blockIdx.y;
     const int64_t n0 = (int64_t)blockIdx.x * GCM_N;
-    // phase 1: thread (j, 8 features): one 4-byte code load, one 8-byte scale load
-    for (int idx = threadIdx.x; idx < ld * (GCM_N / 8); idx += blockDim.x) {
-        const int jj = idx / (GCM_N / 8);
-        const int f0 = (idx - jj * (GCM_N / 8)) * 8;
-        float v[8];
-        if (jj < k) {
-            const int64_t ch = sel[jj];
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(codes_cm + (e * K + ch) * (N / 2) + (n0 + f0) / 2);
-            const uint2 sc = *reinterpret_cast<const uint2 *>(scales_cm + (e * (K / 16) + (ch >> 4)) * N + n0 + f0);
-            float q[8];
-            e2m1x8_to_f32(w, q);
-            const uint32_t sw[2] = {sc.x, sc.y};
+    if (threadIdx.x < 128) e4[threadIdx.x] = e4m3_to_f32(threadIdx.x);
+    for (int j = threadIdx.x; j < k; j += blockDim.x) ssel[j] = sel[j];
+    __syncthreads();
+    // phase 1: item (channel j, 32 features): 16 B of codes, 32 B of scales;
+    // consecutive threads take consecutive channels, so the 32 shared-memory
+    // stores of an item hit 32 consecutive words across the warp
+    const int groups = GCM_N / 32;
+    for (int idx = threadIdx.x; idx < ld * groups; idx += blockDim.x) {
+        const int jj = idx % ld;
+        const int f0 = (idx / ld) * 32;
+        float v[32];
+        if (jj < k && n0 + f0 < N) {
+            const int64_t ch = ssel[jj];
+            const uint4 w = *reinterpret_cast<const uint4 *>(codes_cm + (e * K + ch) * (N / 2) + (n0 + f0) / 2);
+            const uint4 *sp = reinterpret_cast<const uint4 *>(scales_cm + (e * (K / 16) + (ch >> 4)) * N + n0 + f0);
+            const uint4 s0 = sp[0], s1 = sp[1];
+            const uint32_t cw[4] = {w.x, w.y, w.z, w.w};
+            const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(q[i], e4m3_to_f32((sw[i >> 2] >> (8 * (i & 3))) & 0xFFu));
+            for (int q = 0; q < 4; ++q) {
+                float c8[8];
+                e2m1x8_to_f32(cw[q], c8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int f = q * 8 + i;
+                    v[f] = __fmul_rn(c8[i], e4[(sw[f >> 2] >> (8 * (f & 3))) & 0x7Fu]);
+                }
+            }
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+            for (int f = 0; f < 32; ++f) v[f] = 0.0f;
         }
-        float4 *dst = reinterpret_cast<float4 *>(gtile + jj * GCM_TS + f0);
-        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+        for (int f = 0; f < 32; ++f) gtile[(f0 + f) * ld + jj] = v[f];
     }
     __syncthreads();
-    // phase 2: thread (feature f, 8 channels) writes 16 bytes of out[e, n0 + f, :]
-    for (int idx = threadIdx.x; idx < GCM_N * (ld / 8); idx += blockDim.x) {
-        const int f = idx / (ld / 8);
-        const int j0 = (idx - f * (ld / 8)) * 8;
-        uint32_t pk[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            pk[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(gtile[(j0 + 2 * i) * GCM_TS + f])) |
-                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(gtile[(j0 + 2 * i + 1) * GCM_TS + f])) << 16);
-        *reinterpret_cast<uint4 *>(out + (e * N + n0 + f) * ld + j0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    // phase 2: 16 B (8 channels) per thread, ld / 8 threads per output row:
+    // each row of out[e, n0 + f, :] is written as one contiguous run
+    const int cpr = ld / 8;
+    for (int idx = threadIdx.x; idx < GCM_N * cpr; idx += blockDim.x) {
+        const int f = idx / cpr;
+        const int j0 = (idx - f * cpr) * 8;
+        if (n0 + f >= N) break;                        // rows are monotone in idx
+        const float4 a = *reinterpret_cast<const float4 *>(gtile + f * ld + j0);
+        const float4 b = *reinterpret_cast<const float4 *>(gtile + f * ld + j0 + 4);
+        uint4 o;
+        o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.x)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.y)) << 16);
+        o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.z)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.w)) << 16);
+        o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.x)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.y)) << 16);
+        o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.z)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.w)) << 16);
+        *reinterpret_cast<uint4 *>(out + (e * N + n0 + f) * ld + j0) = o;
     }
 }
 
@@ -854,20 +873,21 @@ extern "C" nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_
                   NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_gather_weight_channels_cm: need N % 64 == 0, K % 64 == 0");
     NVFP4_REQUIRE(k >= 0 && k <= ld && ld % 64 == 0 && ld <= 256 && k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
                   "nvfp4_gather_weight_channels_cm: need 0 <= k <= ld <= 256, ld % 64 == 0");
-    NVFP4_REQUIRE(aligned16(w_sel_dev), NVFP4_ERR_ALIGNMENT, "nvfp4_gather_weight_channels_cm: w_sel alignment");
-    size_t smem = (size_t)ld * GCM_TS * sizeof(float);
+    NVFP4_REQUIRE(aligned16(w_sel_dev) && aligned16(codes_cm_dev) && aligned16(scales_cm_dev), NVFP4_ERR_ALIGNMENT,
+                  "nvfp4_gather_weight_channels_cm: pointers must be 16-byte aligned");
+    size_t smem = (size_t)ld * GCM_N * sizeof(float);
     {
         static bool attr_done[64];
         int dev = 0;
         cudaGetDevice(&dev);
         if (dev >= 0 && dev < 64 && !attr_done[dev]) {
             if (cudaFuncSetAttribute(k_gather_w_channels_cm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)(256 * GCM_TS * sizeof(float))) != cudaSuccess)
+                                     (int)(256 * GCM_N * sizeof(float))) != cudaSuccess)
                 return check_launch("nvfp4_gather_weight_channels_cm: smem attribute");
             attr_done[dev] = true;
         }
     }
-    dim3 grid((unsigned)(N / GCM_N), (unsigned)E);
+    dim3 grid((unsigned)((N + GCM_N - 1) / GCM_N), (unsigned)E);
     k_gather_w_channels_cm<<<grid, 256, smem, (cudaStream_t)stream>>>(codes_cm_dev, scales_cm_dev, N, K, sel_dev, k,
                                                                     ld, (__nv_bfloat16 *)w_sel_dev);
     return check_launch("k_gather_w_channels_cm");
