@@ -1,13 +1,18 @@
 // route.cu -- MoE top-k routing and the expert-grouped routed-row layout.
 //
-//   k_route_topk    one warp per token: k_r rounds of warp argmax over the E
-//                   logits (equal logits: lower expert), softmax over the
-//                   selected logits, per-expert counts (atomics).
-//   k_route_assign  one CTA per expert: padded segment offset (segments are
-//                   multiples of 128 or 256 rows, the GEMM's tile height) from the
-//                   counts, then a block-wide scan over tokens in ascending
-//                   order assigns each (token, slot) routed to the expert its
-//                   row; writes dst_row, row_token, row_gate and the padding.
+//   k_route_topk   one warp per token, 32 tokens per CTA ("routing block"):
+//                  k_r rounds of warp argmax over the E logits (equal logits:
+//                  lower expert), softmax over the selected logits; the
+//                  block's per-expert counts in shared memory -> blkcnt.
+//   k_route_scan   one warp per expert: an exclusive scan of its counts over
+//                  the routing blocks, and the expert's total.
+//   k_route_place  one CTA (32 warps) per routing block: the padded segment
+//                  starts from the totals (segments are multiples of 128 or 256
+//                  rows, the GEMM's tile height; CTA 0 also writes offsets and
+//                  the padding rows' gates); each warp takes experts in turn
+//                  and gives every (token, slot) routed to that expert its row
+//                  = segment start + earlier blocks' count + rank in the block
+//                  (ballot + popcount over the block's tokens in order).
 // Rows inside an expert's segment are in ascending token order, so the layout
 // is deterministic.
 #include "common.cuh"
@@ -18,125 +23,188 @@ namespace nvfp4 {
 
 constexpr int MAX_EXPERTS = 256;
 constexpr int MAX_TOPK = 8;
+constexpr int RB = 32;                   // tokens per routing block (one warp per token)
 
-__global__ void __launch_bounds__(256) k_route_topk(const float *__restrict__ logits, int64_t T, int E, int kr,
+__global__ void __launch_bounds__(1024) k_route_topk(const float *__restrict__ logits, int64_t T, int E, int kr,
                                                     int32_t *__restrict__ topk_idx, float *__restrict__ topk_gate,
-                                                    int32_t *__restrict__ counts)
+                                                    int32_t *__restrict__ blkcnt)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= T) return;
-    float l[MAX_EXPERTS / 32];
+    __shared__ int cnt[MAX_EXPERTS];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    for (int tt = warp; tt < RB; tt += (int)(blockDim.x >> 5)) {
+        const int64_t t = (int64_t)blockIdx.x * RB + tt;
+        if (t >= T) break;                                    // warp-uniform
+        const int nslots = (E + 31) >> 5;                    // populated 32-expert slots
+        float l[MAX_EXPERTS / 32];
 #pragma unroll
-    for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-        int e = lane + 32 * i;
-        l[i] = (e < E) ? logits[t * E + e] : -INFINITY;
-    }
-    unsigned taken = 0;      // bit i: expert lane + 32 i already selected
-    float sel_l[MAX_TOPK];   // fully unrolled below: stays in registers
-    int sel_e[MAX_TOPK];
-#pragma unroll
-    for (int j = 0; j < MAX_TOPK; ++j) {
-        sel_l[j] = -INFINITY;
-        sel_e[j] = 0;
-        if (j < kr) {
-            float bv = -INFINITY;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-                int e = lane + 32 * i;
-                if (e < E && !((taken >> i) & 1u)) {
-                    if (be == 0x7fffffff || l[i] > bv) { bv = l[i]; be = e; }
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
-            }
-            sel_l[j] = bv;
-            sel_e[j] = be;
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+            int e = lane + 32 * i;
+            l[i] = (i < nslots && e < E) ? logits[t * E + e] : -INFINITY;
         }
-    }
-    if (lane == 0) {
-        const float mx = sel_l[0];
-        float z = 0.0f;
-        float ex[MAX_TOPK];
+        unsigned taken = 0;      // bit i: expert lane + 32 i already selected
+        float sel_l[MAX_TOPK];   // fully unrolled below: stays in registers
+        int sel_e[MAX_TOPK];
 #pragma unroll
         for (int j = 0; j < MAX_TOPK; ++j) {
-            ex[j] = j < kr ? expf(sel_l[j] - mx) : 0.0f;
-            z += ex[j];
-        }
-#pragma unroll
-        for (int j = 0; j < MAX_TOPK; ++j) {
+            sel_l[j] = -INFINITY;
+            sel_e[j] = 0;
             if (j < kr) {
-                topk_idx[t * kr + j] = sel_e[j];
-                topk_gate[t * kr + j] = ex[j] / z;
-                atomicAdd(counts + sel_e[j], 1);
+                float bv = -INFINITY;
+                int be = 0x7fffffff;
+#pragma unroll
+                for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+                    if (i >= nslots) break;
+                    int e = lane + 32 * i;
+                    if (e < E && !((taken >> i) & 1u)) {
+                        if (be == 0x7fffffff || l[i] > bv) { bv = l[i]; be = e; }
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                    if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
+                }
+                sel_l[j] = bv;
+                sel_e[j] = be;
+                if ((be & 31) == lane) taken |= 1u << (be >> 5);
             }
         }
-    }
-}
-
-__global__ void __launch_bounds__(1024) k_route_assign(const int32_t *__restrict__ topk_idx,
-                                                       const float *__restrict__ topk_gate, int64_t T, int E, int kr,
-                                                       const int32_t *__restrict__ counts, int align,
-                                                       int32_t *__restrict__ offsets, int32_t *__restrict__ dst_row,
-                                                       int32_t *__restrict__ row_token, float *__restrict__ row_gate)
-{
-    __shared__ int s_base, s_cnt, s_running;
-    __shared__ int warp_sums[32];
-    const int e = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) {
-        int base = 0, total = 0;
-        for (int i = 0; i < E; ++i) {
-            int padded = (counts[i] + align - 1) / align * align;
-            if (i < e) base += padded;
-            total += padded;
+        // softmax over the selected logits: lane j < k_r handles slot j; z is
+        // summed in slot order (the same order as a serial loop)
+        float my_l = sel_l[0];
+        int my_e = sel_e[0];
+#pragma unroll
+        for (int j = 1; j < MAX_TOPK; ++j)
+            if (lane == j) { my_l = sel_l[j]; my_e = sel_e[j]; }
+        const float ex = lane < kr ? expf(my_l - sel_l[0]) : 0.0f;
+        float z = 0.0f;
+#pragma unroll
+        for (int j = 0; j < MAX_TOPK; ++j) z += __shfl_sync(0xffffffffu, ex, j);
+        if (lane < kr) {
+            topk_idx[t * kr + lane] = my_e;
+            topk_gate[t * kr + lane] = ex / z;
+            atomicAdd(&cnt[my_e], 1);
         }
-        s_base = base;
-        s_cnt = counts[e];
-        s_running = 0;
-        offsets[e] = base;
-        if (e == E - 1) offsets[E] = total;
     }
     __syncthreads();
-    const int base = s_base;
-    for (int64_t t0 = 0; t0 < T; t0 += blockDim.x) {
-        int64_t t = t0 + tid;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) blkcnt[(int64_t)i * gridDim.x + blockIdx.x] = cnt[i];   // [E][nblk]
+}
+
+// One warp per expert (4 per CTA).  blkcnt [E x nblk] (expert-major, so each
+// expert's counts are contiguous) is turned in place into each block's
+// exclusive prefix within its expert; tot[e] = the expert's routed rows.
+__global__ void __launch_bounds__(128) k_route_scan(int32_t *__restrict__ blkcnt, int nblk, int E,
+                                                    int32_t *__restrict__ tot)
+{
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (e >= E) return;                                      // warp-uniform
+    int running = 0;
+    for (int b0 = 0; b0 < nblk; b0 += 32 * 8) {
+        // lane l takes 8 consecutive blocks: independent loads, a
+        // thread-local prefix, then a warp scan of the lane sums
+        int c[8], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int b = b0 + lane * 8 + i;
+            c[i] = b < nblk ? blkcnt[(int64_t)e * nblk + b] : 0;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sum += c[i];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int pre = running + incl - sum;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int b = b0 + lane * 8 + i;
+            if (b < nblk) blkcnt[(int64_t)e * nblk + b] = pre;
+            pre += c[i];
+        }
+        running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) tot[e] = running;
+}
+
+__global__ void __launch_bounds__(1024) k_route_place(const int32_t *__restrict__ topk_idx,
+                                                     const float *__restrict__ topk_gate, int64_t T, int E, int kr,
+                                                     const int32_t *__restrict__ blkoff,
+                                                     const int32_t *__restrict__ tot, int align,
+                                                     int32_t *__restrict__ offsets,
+                                                     int32_t *__restrict__ dst_row, int32_t *__restrict__ row_token,
+                                                     float *__restrict__ row_gate)
+{
+    __shared__ int32_t sidx[MAX_TOPK * RB];          // [slot][token in block]
+    __shared__ int sbase[MAX_EXPERTS + 1];           // padded segment starts
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = (int)(blockDim.x >> 5);
+    const int64_t t0 = (int64_t)blockIdx.x * RB;
+    const int nt = (int)std::min<int64_t>(RB, T - t0);
+    for (int i = threadIdx.x; i < MAX_TOPK * RB; i += blockDim.x) {
+        const int j = i / RB, tt = i - j * RB;
+        sidx[i] = (j < kr && tt < nt) ? topk_idx[(t0 + tt) * kr + j] : -1;
+    }
+    if (warp == 0) {
+        // padded exclusive scan of the expert totals: lane l takes 8 experts
+        int c[MAX_EXPERTS / 32], sum = 0;
+#pragma unroll
+        for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+            const int e = lane * (MAX_EXPERTS / 32) + i;
+            c[i] = e < E ? (tot[e] + align - 1) / align * align : 0;
+            sum += c[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int pre = incl - sum;
+#pragma unroll
+        for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+            const int e = lane * (MAX_EXPERTS / 32) + i;
+            if (e < E) sbase[e] = pre;
+            pre += c[i];
+        }
+        if (lane == 31) sbase[E] = incl;                     // total padded rows
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = sbase[e];
+        // gates of the padding rows at the end of each segment
+        for (int i = threadIdx.x; i < E * align; i += blockDim.x) {
+            const int e = i / align, r = sbase[e] + tot[e] + (i - e * align);
+            if (r < sbase[e + 1]) row_gate[r] = 0.0f;
+        }
+    }
+    // the warp's experts are e = warp + nwarps * i; lane i prefetches the
+    // row base of expert i of the warp (segment start + earlier blocks)
+    int mybase = 0;
+    {
+        const int e = warp + nwarps * lane;
+        if (e < E) mybase = sbase[e] + blkoff[(int64_t)e * gridDim.x + blockIdx.x];
+    }
+    static_assert(RB == 32, "one ballot per expert covers the block");
+    for (int i = 0, e = warp; e < E; ++i, e += nwarps) {
+        const int run = __shfl_sync(0xffffffffu, mybase, i);
+        const int tt = lane;
         int slot = -1;
-        if (t < T) {
-            for (int j = 0; j < kr; ++j)
-                if (topk_idx[t * kr + j] == e) slot = j;
-        }
-        unsigned ballot = __ballot_sync(0xffffffffu, slot >= 0);
-        int within = __popc(ballot & ((1u << lane) - 1u));
-        if (lane == 0) warp_sums[warp] = __popc(ballot);
-        __syncthreads();
-        int before = 0, chunk_total = 0;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-            int s = warp_sums[w];
-            if (w < warp) before += s;
-            chunk_total += s;
-        }
+#pragma unroll
+        for (int j = 0; j < MAX_TOPK; ++j)
+            if (sidx[j * RB + tt] == e) slot = j;
+        const unsigned bal = __ballot_sync(0xffffffffu, slot >= 0);
         if (slot >= 0) {
-            int row = base + s_running + before + within;
+            const int row = run + __popc(bal & ((1u << lane) - 1u));
+            const int64_t t = t0 + tt;
             dst_row[t * kr + slot] = row;
             row_token[row] = (int32_t)t;
             row_gate[row] = topk_gate[t * kr + slot];
         }
-        __syncthreads();
-        if (tid == 0) s_running += chunk_total;
-        __syncthreads();
-    }
-    const int cnt = s_cnt;
-    const int padded = (cnt + align - 1) / align * align;
-    for (int i = cnt + tid; i < padded; i += blockDim.x) {
-        row_token[base + i] = -1;
-        row_gate[base + i] = 0.0f;
     }
 }
 
@@ -182,9 +250,9 @@ extern "C" nvfp4_status moe_gather_rows_bf16(const void *x_dev, int64_t T, int64
 
 extern "C" size_t moe_route_workspace_size(int64_t T, int32_t E)
 {
-    (void)T;
-    if (E <= 0) return 0;
-    return (size_t)((E * 4 + 255) / 256 * 256);
+    if (E <= 0 || T < 0) return 0;
+    const int64_t nblk = std::max<int64_t>(1, (T + RB - 1) / RB);
+    return (size_t)(((nblk + 1) * E * 4 + 255) / 256 * 256);          // block counts [E x nblk] + totals [E]
 }
 
 extern "C" nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E, int32_t k_r,
@@ -206,16 +274,23 @@ extern "C" nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E,
     size_t need = moe_route_workspace_size(T, E);
     NVFP4_REQUIRE(workspace && workspace_bytes >= need, NVFP4_ERR_WORKSPACE,
                   "moe_route: workspace of %zu bytes required", need);
-    int32_t *counts = reinterpret_cast<int32_t *>(workspace);
-    if (cudaMemsetAsync(counts, 0, (size_t)E * 4, st) != cudaSuccess) return check_launch("moe_route memset");
+    int32_t *blkcnt = reinterpret_cast<int32_t *>(workspace);
+    const int nblk = (int)((T + RB - 1) / RB);
     if (cudaMemsetAsync(row_token_dev, 0xFF, (size_t)M_pad_max * 4, st) != cudaSuccess)
         return check_launch("moe_route memset");
-    if (T > 0) {
-        k_route_topk<<<(unsigned)((T + 7) / 8), 256, 0, st>>>(logits_dev, T, E, k_r, topk_idx_dev, topk_gate_dev,
-                                                             counts);
+    if (nblk > 0) {
+        k_route_topk<<<(unsigned)nblk, 1024, 0, st>>>(logits_dev, T, E, k_r, topk_idx_dev, topk_gate_dev, blkcnt);
         if (check_launch("k_route_topk") != NVFP4_OK) return NVFP4_ERR_CUDA;
     }
-    k_route_assign<<<(unsigned)E, 1024, 0, st>>>(topk_idx_dev, topk_gate_dev, T, E, k_r, counts, seg_align, offsets_dev,
-                                                dst_row_dev, row_token_dev, row_gate_dev);
-    return check_launch("k_route_assign");
+    int32_t *tot = blkcnt + (int64_t)nblk * E;
+    if (nblk == 0) {
+        // no tokens: every expert segment is empty
+        if (cudaMemsetAsync(offsets_dev, 0, (size_t)(E + 1) * 4, st) != cudaSuccess) return check_launch("moe_route memset");
+        return NVFP4_OK;
+    }
+    k_route_scan<<<(unsigned)((E + 3) / 4), 128, 0, st>>>(blkcnt, nblk, E, tot);
+    if (check_launch("k_route_scan") != NVFP4_OK) return NVFP4_ERR_CUDA;
+    k_route_place<<<(unsigned)nblk, 1024, 0, st>>>(topk_idx_dev, topk_gate_dev, T, E, k_r, blkcnt, tot, seg_align,
+                                                  offsets_dev, dst_row_dev, row_token_dev, row_gate_dev);
+    return check_launch("k_route_place");
 }
