@@ -41,6 +41,22 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FP4_PER_BF16 = 4.0          # nominal dense FP4 : BF16 tensor-core ratio (9 : 2.25 PFLOP/s)
 QUANT_BYTES_PER_ELEM = 2.5625   # 2 B bf16 read + 0.5 B codes + 1/16 B scale written
 
+# DRAM traffic of k_moe_gemm per launch (dram__bytes_read.sum + dram__bytes_write.sum,
+# averaged over the gate/up and down launches of one step) from the ncu capture
+# summarised in profiles/k_moe_gemm_moe_t16384_e128.md, valid only for the kernel
+# sources it was taken on (sha256 of gemm.cu + ptx.cuh + common.cuh).
+GEMM_TRAFFIC = {"bytes_per_launch": None, "sources_sha256": None}
+
+
+def gemm_traffic():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "ptx.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "quantization_nvfp4_quantize_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    ok = GEMM_TRAFFIC["sources_sha256"] == h.hexdigest()
+    return GEMM_TRAFFIC["bytes_per_launch"] if ok else None
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -245,7 +261,8 @@ def run_ours(args):
                    "l2": "inputs larger than L2 (NVFP4 weights 1.36 GB)", "parallelism": f"replicas x{ws}"},
         "roofline": {"bound": "tensor", "kernel": "k_moe_gemm",
                      "achieved": round(gemm_fp4_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(gemm_fp4_tflops / fp4_peak, 4), "traffic": None,
+                     "frac": round(gemm_fp4_tflops / fp4_peak, 4), "traffic": gemm_traffic(),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_source": f"{p['source']} bf16 sustained x{FP4_PER_BF16:g} (nominal FP4:BF16)",
                      "achieved_incl_rac": round(gemm_all_tflops, 1),
                      "gemm_ms_per_step": round(gemm_ms / args.steps, 4), "launches_per_step": n_gemm // args.steps},
@@ -257,7 +274,7 @@ def run_ours(args):
         "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=8)
+        out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=40)
     if rank == 0:
         print(json.dumps(out), flush=True)
     return out
@@ -399,29 +416,74 @@ def run_ours_w4a16(args):
 
 def run_e2e(layer, x, logits, args, dev):
     """Same metric through the public API with host buffers: every step copies
-    X and the router logits from pinned host memory and Y back."""
+    its X and router logits from pinned host memory to the device and reads
+    its Y back into pinned host memory.  Steps are pipelined the way a serving
+    loop would run them: inputs of step i+1 travel host->device on one copy
+    stream and Y of step i-1 device->host on another (PCIe is full duplex)
+    while step i computes; Y is staged device-to-device so the next step can
+    reuse the layer's output buffer.  Two buffers per direction; events order
+    every reuse."""
     import torch
-    xh = x.cpu().pin_memory()
-    lh = logits.cpu().pin_memory()
-    yh = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
-    xd = torch.empty_like(x)
-    ld = torch.empty_like(logits)
-    stream = torch.cuda.current_stream(dev)
-    steps = max(1, args.steps // 2)
-    for _ in range(2):
-        xd.copy_(xh, non_blocking=True)
-        ld.copy_(lh, non_blocking=True)
-        yh.copy_(layer.forward(xd, ld), non_blocking=True)
+    steps = max(2, args.steps // 2)
+    xh = [x.cpu().pin_memory() for _ in range(2)]
+    lh = [logits.cpu().pin_memory() for _ in range(2)]
+    yh = [torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(x) for _ in range(2)]
+    ld = [torch.empty_like(logits) for _ in range(2)]
+    ys = [torch.empty_like(layer.y) for _ in range(2)]
+    comp = torch.cuda.current_stream(dev)
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+
+    def run(n, start):
+        in_ready = [ev(), ev()]      # inputs of buffer b landed
+        in_free = [None, None]       # the step that read buffer b has finished
+        out_ready = [ev(), ev()]     # ys[b] holds a finished Y
+        out_free = [None, None]      # the read-back of ys[b] has finished
+        s_in.wait_event(start)       # no copy starts before the timed region
+        s_out.wait_event(start)
+        with torch.cuda.stream(s_in):
+            xd[0].copy_(xh[0], non_blocking=True)
+            ld[0].copy_(lh[0], non_blocking=True)
+            in_ready[0].record(s_in)
+        for i in range(n):
+            b = i & 1
+            if i + 1 < n:            # prefetch the next step's inputs
+                nb = (i + 1) & 1
+                with torch.cuda.stream(s_in):
+                    if in_free[nb] is not None:
+                        s_in.wait_event(in_free[nb])
+                    xd[nb].copy_(xh[nb], non_blocking=True)
+                    ld[nb].copy_(lh[nb], non_blocking=True)
+                    in_ready[nb].record(s_in)
+            comp.wait_event(in_ready[b])
+            y = layer.forward(xd[b], ld[b])
+            if out_free[b] is not None:
+                comp.wait_event(out_free[b])
+            ys[b].copy_(y, non_blocking=True)
+            in_free[b] = ev()
+            in_free[b].record(comp)
+            out_ready[b].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(out_ready[b])
+                yh[b].copy_(ys[b], non_blocking=True)
+                out_free[b] = ev()
+                out_free[b].record(s_out)
+        for f in out_free:           # the end event follows every read-back
+            if f is not None:
+                comp.wait_event(f)
+
+    w = torch.cuda.Event()
+    w.record(comp)
+    run(2, w)                        # warm-up
     torch.cuda.synchronize()
     barrier()
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(steps):
-        xd.copy_(xh, non_blocking=True)
-        ld.copy_(lh, non_blocking=True)
-        yh.copy_(layer.forward(xd, ld), non_blocking=True)
-    e.record(stream)
+    s.record(comp)
+    run(steps, s)
+    e.record(comp)
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e), dev)
     from quantization_nvfp4_quantize_b200 import workloads as wl
@@ -429,8 +491,9 @@ def run_e2e(layer, x, logits, args, dev):
     fl = wl.flops(cfg)
     ws = dist_env()[0]
     return {"value": round((fl["fp4"] + fl["rac"]) * steps * ws / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": xh.numel() * xh.element_size() + lh.numel() * lh.element_size(),
-            "d2h_bytes_per_step": yh.numel() * yh.element_size()}
+            "h2d_bytes_per_step": xh[0].numel() * xh[0].element_size() + lh[0].numel() * lh[0].element_size(),
+            "d2h_bytes_per_step": yh[0].numel() * yh[0].element_size(),
+            "pipelined": "H2D of step i+1 and D2H of step i-1 overlap step i (two copy streams)"}
 
 
 # --------------------------------------------------------------- CPU oracle

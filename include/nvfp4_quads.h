@@ -221,6 +221,8 @@ NVFP4_API nvfp4_status nvfp4_qdq_weights(const void *w_dev, int64_t G, int64_t r
  *                and for rows >= offsets[E].
  *   row_gate_dev float32 [M_pad_max]: gate of each routed row (0 for padding).
  *   M_pad_max    >= T*k_r + E*(seg_align-1) rounded up to seg_align.
+ * T may be 0 (the per-token arrays may then be NULL): every segment is empty.
+ * workspace: moe_route_workspace_size(T, E) bytes (per-block expert counts).
  * -------------------------------------------------------------------------- */
 NVFP4_API size_t moe_route_workspace_size(int64_t T, int32_t E);
 

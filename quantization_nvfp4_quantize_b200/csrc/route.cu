@@ -262,8 +262,9 @@ extern "C" nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E,
                                   void *workspace, size_t workspace_bytes, void *stream)
 {
     cudaStream_t st = (cudaStream_t)stream;
-    NVFP4_REQUIRE(logits_dev && topk_idx_dev && topk_gate_dev && offsets_dev && dst_row_dev && row_token_dev &&
-                  row_gate_dev, NVFP4_ERR_INVALID_ARG, "moe_route: null pointer");
+    NVFP4_REQUIRE(offsets_dev && row_token_dev && row_gate_dev &&
+                  (T == 0 || (logits_dev && topk_idx_dev && topk_gate_dev && dst_row_dev)), NVFP4_ERR_INVALID_ARG,
+                  "moe_route: null pointer");
     NVFP4_REQUIRE(T >= 0 && E >= 1 && E <= MAX_EXPERTS && k_r >= 1 && k_r <= MAX_TOPK && k_r <= E,
                   NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_route: need 1 <= E <= 256, 1 <= k_r <= min(8, E)");
     NVFP4_REQUIRE(seg_align == 128 || seg_align == 256, NVFP4_ERR_INVALID_ARG, "moe_route: seg_align must be 128 or 256");

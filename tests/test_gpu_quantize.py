@@ -158,7 +158,8 @@ def test_qdq_weights_parity(cuda, G, rows, cols):
 
 
 @pytest.mark.parametrize("T,E,kr,align", [(512, 8, 2, 128), (1000, 128, 8, 128), (64, 1, 1, 128), (3, 16, 4, 128),
-                                          (4096, 256, 8, 128), (1000, 128, 8, 256), (700, 8, 2, 256)])
+                                          (4096, 256, 8, 128), (1000, 128, 8, 256), (700, 8, 2, 256),
+                                          (0, 8, 2, 256), (33, 3, 3, 256), (16384, 128, 8, 256)])
 def test_route_parity(cuda, T, E, kr, align):
     rng = np.random.default_rng(T + E)
     logits = rng.standard_normal((T, E)).astype(np.float32)
@@ -181,12 +182,16 @@ def test_route_parity(cuda, T, E, kr, align):
         toks = np.nonzero((idx == e).any(axis=1))[0]
         assert np.array_equal(seg[: counts[e]], toks)            # ascending tokens
         assert np.all(seg[counts[e]:] == -1)
+        assert np.all(rg[off[e] + counts[e]:off[e + 1]] == 0)   # padding rows carry no gate
     assert np.all(tok[off[E]:] == -1)
-    for t in range(T):
-        for j in range(kr):
-            d = dst[t, j]
-            assert tok[d] == t and off[idx[t, j]] <= d < off[idx[t, j] + 1]
-            assert rg[d] == r.topk_gate[t, j].item()
+    if T:
+        tt = np.repeat(np.arange(T), kr)
+        d = dst.reshape(-1)
+        e = idx.reshape(-1)
+        assert np.array_equal(tok[d], tt)
+        assert np.all((off[e] <= d) & (d < off[e + 1]))
+        assert np.array_equal(rg[d], r.topk_gate.cpu().numpy().reshape(-1))
+        assert len(np.unique(d)) == T * kr
 
 
 def test_gather_weight_channels(cuda):
