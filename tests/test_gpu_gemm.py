@@ -147,3 +147,31 @@ def test_dense_layer_config(cuda):
     rho = oracle.rac_residual(qx.resid, qx.s_t, S)
     want = oracle.w4a4_rac_matmul(qx.xhat, qx.s_t, rho, S, oracle.quantize(wn).xhat)
     assert rel_fro(y, want) <= TOL
+
+
+@pytest.mark.parametrize("align", [128, 256])
+def test_gemm_no_routed_rows(cuda, align):
+    """T = 0: every expert segment is empty, the GEMMs write nothing (the
+    scatter target keeps its contents, store rows stay untouched)."""
+    rng = np.random.default_rng(17)
+    E, N, K = 4, 256, 256
+    logits = torch.empty(0, E, dtype=torch.float32, device=cuda)
+    r = api.route(logits, 2, seg_align=align)
+    assert r.offsets.cpu().numpy().tolist() == [0] * (E + 1)
+    w = gen(rng, (E, N, K), 0.05)
+    _, s_w, c_w, sf_w = api.qdq_weights(to_bf16_dev(w, cuda), want_qdq=False, want_packed=True)
+    a_codes = torch.zeros(r.m_pad_max, K // 2, dtype=torch.uint8, device=cuda)
+    a_scales = torch.zeros(api.scale_bytes(r.m_pad_max, K), dtype=torch.uint8, device=cuda)
+    s_a = torch.ones(1, dtype=torch.float32, device=cuda)
+    out = torch.full((r.m_pad_max, N), 7.0, dtype=torch.float32, device=cuda)
+    api.grouped_gemm(a_codes, a_scales, s_a, r.m_pad_max, c_w, sf_w, s_w, N, K, E, r.offsets, seg_align=align,
+                     epilogue=api.EPI_STORE_F32, row_token=r.row_token, row_gate=r.row_gate, out=out)
+    y = torch.full((1, N), 3.0, dtype=torch.float32, device=cuda)
+    api.grouped_gemm(a_codes, a_scales, s_a, r.m_pad_max, c_w, sf_w, s_w, N, K, E, r.offsets, seg_align=align,
+                     epilogue=api.EPI_SCATTER_ADD_F32, row_token=r.row_token, row_gate=r.row_gate, out=y)
+    a16 = torch.zeros(r.m_pad_max, K, dtype=torch.bfloat16, device=cuda)
+    out16 = torch.full((r.m_pad_max, N), 5.0, dtype=torch.float32, device=cuda)
+    api.bf16_grouped_gemm(a16, r.m_pad_max, to_bf16_dev(w, cuda), N, K, E, r.offsets, seg_align=align,
+                          epilogue=api.EPI_STORE_F32, row_token=r.row_token, row_gate=r.row_gate, out=out16)
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0) and torch.all(y == 3.0) and torch.all(out16 == 5.0)
