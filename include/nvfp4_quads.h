@@ -307,7 +307,14 @@ NVFP4_API nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_d
  *                   <= 256; rho_dev bf16 [M_pad_max x rac_ld] and
  *                   w_sel_dev bf16 [E x N x rac_ld].
  * Shapes: K % 256 == 0, N % 256 == 0 (SWIGLU: I % 128 == 0), M_pad_max a
- * multiple of seg_align, E <= 256.  Persistent kernel: one CTA per SM.
+ * multiple of seg_align, E <= 256; pointers 16-byte aligned.  Persistent
+ * kernel: one CTA per SM (seg_align 256: one 2-CTA cluster per SM pair); the
+ * tile count is read from offsets[E] on the device (no host sync).
+ * Errors: argument, shape and alignment errors are returned synchronously;
+ * a device wait that exceeds its bound (1 s) writes NVFP4_ERR_TIMEOUT to
+ * dev_status (if given) and the kernel exits cleanly.  Tuning only: the
+ * environment variable NVFP4_GEMM_NGROUP (a divisor of the n-tile count)
+ * overrides how many n-tiles run as one group in the tile order.
  * -------------------------------------------------------------------------- */
 typedef enum {
     MOE_EPI_STORE_F32 = 0,
