@@ -274,7 +274,7 @@ def run_ours(args):
         "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=40)
+        out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=64)
     if rank == 0:
         print(json.dumps(out), flush=True)
     return out
