@@ -55,7 +55,8 @@
 // columns), B's in the next 32 (4 x 8 columns); at most 5 stages.
 // Every mbarrier wait is bounded (1 s); on expiry the kernel records
 // NVFP4_ERR_TIMEOUT, all roles stop, in-flight copies and MMAs are drained
-// (bounded) and TMEM is freed before exit.  No TMA load uses multicast.
+// (bounded) and TMEM is freed before exit.  Every TMA load writes only the
+// issuing CTA's own shared memory.
 #include "common.cuh"
 #include "ptx.cuh"
 

@@ -1,6 +1,6 @@
 // ptx.cuh -- thin inline-PTX wrappers for the sm_100a features the grouped
-// GEMM uses: mbarriers, TMA (cp.async.bulk.tensor, never with cluster
-// multicast), bulk copies, and the 5th-generation tensor core (tcgen05: TMEM
+// GEMM uses: mbarriers, TMA tensor loads (each into the issuing CTA's own
+// shared memory), bulk copies, and the 5th-generation tensor core (tcgen05: TMEM
 // allocation, shared-memory -> TMEM copies of scale factors, block-scaled FP4
 // and BF16 MMAs, commits, TMEM loads).  Written from the public PTX ISA.
 #pragma once
