@@ -45,7 +45,7 @@ QUANT_BYTES_PER_ELEM = 2.5625   # 2 B bf16 read + 0.5 B codes + 1/16 B scale wri
 # averaged over the gate/up and down launches of one step) from the ncu capture
 # summarised in profiles/k_moe_gemm_moe_t16384_e128.md, valid only for the kernel
 # sources it was taken on (sha256 of gemm.cu + ptx.cuh + common.cuh).
-GEMM_TRAFFIC = {"bytes_per_launch": 2392299456, "sources_sha256": "a4f420c91fca3957acf96ec9b2c335c2b9e7df09bf2dfff33f8624ddb464d305"}
+GEMM_TRAFFIC = {"bytes_per_launch": 2402440832, "sources_sha256": "abb4d348896f0d6a59bc4890a5ac3c54130350562651dfc2a26f8b946fb6e704"}
 
 
 def gemm_traffic():
