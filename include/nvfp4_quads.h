@@ -238,6 +238,7 @@ NVFP4_API nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E, 
  * scale (e2m1 * sf is exact in bf16):
  *   w_sel[e, n, j] = bf16(e2m1(q_e[n, S_j]) * sf_e[n, S_j/16])  (j < k)
  *   w_sel[e, n, j] = 0                                          (k <= j < ld)
+ * A selected index outside [0, K) also gives a zero column.
  *   codes_dev  uint8 [E x N x K/2], scales_dev swizzled per expert.
  *   w_sel_dev  bf16 [E x N x ld], ld % 64 == 0, k <= ld.
  * -------------------------------------------------------------------------- */

@@ -498,8 +498,8 @@ __global__ void k_gather_w_channels(const uint8_t *__restrict__ codes, const uin
         int64_t en = i / ld;
         int64_t n = en % N, e = en / N;
         float v = 0.0f;
-        if (j < k) {
-            int64_t ch = sel[j];
+        const int64_t ch = j < k ? (int64_t)sel[j] : -1;
+        if (ch >= 0 && ch < K) {                        // channels outside [0, K) give zeros
             uint32_t byte = codes[en * (K >> 1) + (ch >> 1)];
             uint32_t nib = (ch & 1) ? (byte >> 4) : (byte & 15u);
             float q = e2m1x2_to_f32(nib).x;
@@ -570,8 +570,8 @@ __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__r
         const int jj = idx % ld;
         const int f0 = (idx / ld) * 32;
         float v[32];
-        if (jj < k && n0 + f0 < N) {
-            const int64_t ch = ssel[jj];
+        const int64_t ch = jj < k ? (int64_t)ssel[jj] : -1;
+        if (ch >= 0 && ch < K && n0 + f0 < N) {        // channels outside [0, K) give zeros
             const uint4 w = *reinterpret_cast<const uint4 *>(codes_cm + (e * K + ch) * (N / 2) + (n0 + f0) / 2);
             const uint4 *sp = reinterpret_cast<const uint4 *>(scales_cm + (e * (K / 16) + (ch >> 4)) * N + n0 + f0);
             const uint4 s0 = sp[0], s1 = sp[1];

@@ -240,3 +240,23 @@ def test_channel_major_copy_and_gather(cuda, E, N, K, k, ld):
         vals = oracle.e2m1_decode(q) * np.repeat(oracle.e4m3_decode(ref.sf), 16, axis=1)
         want = oracle.f32_to_bf16(vals[:, sel].astype(np.float32))
         assert np.array_equal(np_u16(b)[e, :, :k], want)
+
+
+def test_gather_out_of_range_channels_give_zero_columns(cuda):
+    """Channel indices outside [0, K) give zero columns in both weight
+    gathers; the valid columns are unchanged."""
+    rng = np.random.default_rng(19)
+    E, N, K, k, ld = 2, 128, 256, 6, 64
+    w = oracle.f32_to_bf16(rng.standard_normal((E, N, K)).astype(np.float32) * 0.02)
+    _, s_t, codes, scales = api.qdq_weights(to_bf16_dev(w, cuda), want_qdq=False, want_packed=True)
+    codes_cm, scales_cm = api.weights_channel_major(codes, scales, N, K)
+    sel = np.array([3, K, 17, -1, 100, 1 << 20], np.int32)
+    sel_d = torch.from_numpy(sel).to(cuda)
+    a = np_u16(api.gather_weight_channels(codes, scales, N, K, sel_d, k, ld))
+    b = np_u16(api.gather_weight_channels_cm(codes_cm, scales_cm, N, K, sel_d, k, ld))
+    assert np.array_equal(a, b)
+    bad = [1, 3, 5]
+    assert np.all(a[:, :, bad] == 0) and np.all(a[:, :, k:] == 0)
+    good = np.array([3, 17, 100], np.int32)
+    ref = np_u16(api.gather_weight_channels(codes, scales, N, K, torch.from_numpy(good).to(cuda), 3, ld))
+    assert np.array_equal(a[:, :, [0, 2, 4]], ref[:, :, :3])
