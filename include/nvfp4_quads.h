@@ -114,8 +114,8 @@ NVFP4_API int nvfp4_num_sms(void);
  *   s_t_out_dev  float32 [1]: receives s_t (required).
  *   dst_rows_dev optional int32 [M x fanout]: input row r is written to output
  *                rows dst_rows[r*fanout + j] (j < fanout, 1 <= fanout <= 32);
- *                a negative entry skips that copy.  NULL: output row = input
- *                row, fanout 1.
+ *                a negative entry, or one >= M_out, skips that copy.  NULL:
+ *                output row = input row, fanout 1.
  *   M_out        rows of the output arrays (every destination < M_out).
  *   codes_dev    uint8 [M_out x K/2].
  *   scales_dev   uint8 swizzled, ceil(M_out/128)*128*K/16 bytes.

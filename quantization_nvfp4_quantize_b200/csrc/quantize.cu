@@ -82,6 +82,7 @@ struct QuantParams {
     float *s_t_out;                  // per group
     const int32_t *dst_rows;
     int fanout;
+    int64_t M_out;                   // rows of the outputs: destination rows >= M_out are skipped
     uint8_t *codes;
     uint8_t *scales;
     __nv_bfloat16 *qdq;
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
                 // scale words to each destination.
                 if (lane < p.fanout) {
                     const int64_t dst = p.dst_rows[r * p.fanout + lane];
-                    fan[warp][lane] = dst >= 0 ? make_longlong2(dst * (K >> 1), sf_offset(dst, 0, K))
+                    fan[warp][lane] = (dst >= 0 && dst < p.M_out) ? make_longlong2(dst * (K >> 1), sf_offset(dst, 0, K))
                                                : make_longlong2(-1, 0);
                 }
                 __syncwarp();
@@ -449,7 +450,7 @@ __global__ void __launch_bounds__(256) k_rac_residual(
     const __nv_bfloat16 *__restrict__ x, int64_t ldx, int64_t M, int64_t K,
     const int32_t *__restrict__ m_valid, const float *__restrict__ s_t_ptr,
     const int32_t *__restrict__ sel, int k, int ld,
-    const int32_t *__restrict__ dst_rows, int fanout, __nv_bfloat16 *__restrict__ r_sel)
+    const int32_t *__restrict__ dst_rows, int fanout, int64_t M_out, __nv_bfloat16 *__restrict__ r_sel)
 {
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -479,7 +480,7 @@ __global__ void __launch_bounds__(256) k_rac_residual(
         }
         for (int d = 0; d < nd; ++d) {
             int64_t dst = dst_rows ? (int64_t)dst_rows[r * fanout + d] : r;
-            if (dst >= 0) r_sel[dst * ld + j] = outv;
+            if (dst >= 0 && dst < M_out) r_sel[dst * ld + j] = outv;
         }
     }
 }
@@ -737,6 +738,7 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
     p.s_t_out = s_t_out_dev;
     p.dst_rows = dst_rows_dev;
     p.fanout = dst_rows_dev ? fanout : 1;
+    p.M_out = M_out;
     p.codes = codes_dev;
     p.scales = scales_dev;
     p.qdq = nullptr;
@@ -768,7 +770,7 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
             unsigned blocks = (unsigned)((M + 7) / 8);
             k_rac_residual<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, s_t_used,
                                                    sel_dev, rac_k, rac_ld, dst_rows_dev,
-                                                   dst_rows_dev ? fanout : 1, (__nv_bfloat16 *)r_sel_dev);
+                                                   dst_rows_dev ? fanout : 1, M_out, (__nv_bfloat16 *)r_sel_dev);
             if (check_launch("k_rac_residual") != NVFP4_OK) return NVFP4_ERR_CUDA;
         }
     }
@@ -818,6 +820,7 @@ extern "C" nvfp4_status nvfp4_qdq_weights(const void *w_dev, int64_t G, int64_t 
     p.amax_bits = amax_bits;
     p.s_t_out = s_t_dev;
     p.fanout = 1;
+    p.M_out = rows;
     p.codes = codes_dev;
     p.scales = scales_dev;
     p.qdq = (__nv_bfloat16 *)w_qdq_dev;

@@ -260,3 +260,34 @@ def test_gather_out_of_range_channels_give_zero_columns(cuda):
     good = np.array([3, 17, 100], np.int32)
     ref = np_u16(api.gather_weight_channels(codes, scales, N, K, torch.from_numpy(good).to(cuda), 3, ld))
     assert np.array_equal(a[:, :, [0, 2, 4]], ref[:, :, :3])
+
+
+def test_fanout_skips_rows_beyond_m_out(cuda):
+    """Destination rows >= M_out are skipped like negative ones: the outputs'
+    guard rows past M_out keep their contents, the valid copies are exact."""
+    rng = np.random.default_rng(23)
+    M, K, F, m_out, guard = 64, 256, 2, 256, 128
+    x = gen_x(rng, M, K)
+    dst = np.stack([np.arange(M), M + np.arange(M)], axis=1).astype(np.int32)
+    dst[3, 0] = m_out                        # first guard row
+    dst[9, 1] = m_out + 77                   # deep inside the guard
+    out = api.Quantized(
+        codes=torch.full((m_out + guard, K // 2), 0xAB, dtype=torch.uint8, device=cuda),
+        scales=torch.full((api.scale_bytes(m_out + guard, K),), 0xAB, dtype=torch.uint8, device=cuda),
+        s_t=torch.empty(1, dtype=torch.float32, device=cuda),
+        score=torch.empty(K, dtype=torch.float64, device=cuda),
+        sel=torch.empty(16, dtype=torch.int32, device=cuda),
+        r_sel=torch.full((m_out + guard, 64), 7.0, dtype=torch.bfloat16, device=cuda))
+    api.quantize(to_bf16_dev(x, cuda), rac_k=16, dst_rows=torch.from_numpy(dst).to(cuda), fanout=F, m_out=m_out,
+                 out=out)
+    torch.cuda.synchronize()
+    codes = out.codes.cpu().numpy()
+    assert np.all(codes[m_out:] == 0xAB)
+    assert np.all(out.scales.cpu().numpy()[api.scale_bytes(m_out, K):] == 0xAB)
+    assert torch.all(out.r_sel[m_out:].float() == 7.0)
+    ref = oracle.quantize(x)
+    for r in range(M):
+        for j in range(F):
+            d = dst[r, j]
+            if d < m_out:
+                assert np.array_equal(codes[d], ref.codes[r])
