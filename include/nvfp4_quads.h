@@ -294,7 +294,9 @@ NVFP4_API nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_d
  *                        (the value nvfp4_quantize's amax_in_dev takes).
  *   MOE_EPI_SCATTER_ADD_F32  out f32 [T x ld_out]:
  *                        out[row_token[r], n] += row_gate[r] * y[r,n]
- *                        (atomic; the caller zeroes out first).
+ *                        (atomic; the caller zeroes out first).  Every
+ *                        row_token >= 0 must be a row of out (< T), as
+ *                        moe_route's are; the kernel does not check it.
  *
  *   a_codes_dev/a_scales_dev  NVFP4 A, rows in routed order, M_pad_max rows.
  *   a_s_t_dev       float32 [1].
