@@ -44,16 +44,45 @@ QUANT_BYTES_PER_ELEM = 2.5625   # 2 B bf16 read + 0.5 B codes + 1/16 B scale wri
 # DRAM traffic of k_moe_gemm per launch (dram__bytes_read.sum + dram__bytes_write.sum,
 # averaged over the gate/up and down launches of one step) from the ncu capture
 # summarised in profiles/k_moe_gemm_moe_t16384_e128.md, valid only for the kernel
-# sources it was taken on (sha256 of gemm.cu + ptx.cuh + common.cuh).
-GEMM_TRAFFIC = {"bytes_per_launch": 2402440832, "sources_sha256": "abb4d348896f0d6a59bc4890a5ac3c54130350562651dfc2a26f8b946fb6e704"}
+# code it was taken on: sha256 of gemm.cu + ptx.cuh + common.cuh with comments
+# removed and whitespace collapsed (a comment edit leaves the kernel, and the
+# figure, as is).
+GEMM_TRAFFIC = {"bytes_per_launch": 2402440832, "sources_sha256": "620d862eca54259eefb401c1710b09ed01b8f62a011824243bf4e7ada3bb76c6"}
+
+
+def _code_only(src: str) -> str:
+    """C/C++ source without comments, whitespace runs collapsed (string literals kept)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == '"' or c == "'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif c.isspace():
+            if out and out[-1] != " ":
+                out.append(" ")                  # a run of whitespace -> one space
+            i += 1
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
 
 
 def gemm_traffic():
     import hashlib
     h = hashlib.sha256()
     for f in ("gemm.cu", "ptx.cuh", "common.cuh"):
-        with open(os.path.join(ROOT, "quantization_nvfp4_quantize_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "quantization_nvfp4_quantize_b200", "csrc", f)) as fh:
+            h.update(_code_only(fh.read()).encode())
     ok = GEMM_TRAFFIC["sources_sha256"] == h.hexdigest()
     return GEMM_TRAFFIC["bytes_per_launch"] if ok else None
 

@@ -8,8 +8,12 @@
 //           x 256 features: each CTA holds 128 rows of A, half of B (128
 //           features) and the scale factors its half needs; the even CTA
 //           ("leader") issues every scale-factor copy and MMA for both SMs.
-//           Each scale copy and each MMA then covers twice the work, and each
-//           SM stages half the B bytes.  Expert segments padded to 256 rows.
+//           Per SM the MMA and scale-copy work per stage is unchanged, but
+//           each SM stages only half the B bytes, which leaves room for a
+//           fifth stage.  Expert segments padded to 256 rows.
+// The same kernel serves the BF16 grouped GEMM (moe_bf16_grouped_gemm): no
+// FP4 stage, K / 64 BF16 stages over the whole contraction, unit tensor
+// scales.
 //
 // Warps (384 threads per CTA):
 //   warps 0, 2  TMA producers (one lane each): per 256-element K step warp 0
@@ -43,7 +47,9 @@
 //               bf16 / router-weighted scatter-add into the token-major
 //               output.
 // Tiles never span two experts (segments are multiples of the tile height);
-// the tile count comes from the device-side offsets (no host sync).
+// the tile count comes from the device-side offsets (no host sync).  Tile
+// order: m-major, except that the scatter-add epilogue runs the n-tiles in
+// groups of 2, so the band of token rows being reduced into stays in L2.
 //
 // Shared memory: a ring of stages (single 54 KB, pair 38 KB: 4 / 5 stages for
 // the bf16 epilogue, 3 / 5 for the f32 ones) plus, for the f32 epilogues, a
