@@ -103,3 +103,57 @@ def test_bf16_rounding_matches_torch():
     ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(ours, ref)
     assert np.array_equal(oracle.bf16_to_f32(ours), torch.from_numpy(ours.view(np.int16)).view(torch.bfloat16).float().numpy())
+
+
+# ---------------------------------------------------- scale-factor byte layout
+# Structural pins of oracle.swizzle_scales / unswizzle_scales.  The layout
+# itself is pinned on the GPU, where the tensor cores consume it and the GEMM
+# matches the oracle's products.  Here: it is a bijection onto the padded
+# buffer, its inverse is exact, padding rows are zero, and it has the two
+# properties the kernels rely on (a row's four scales of one 64-element block
+# group are one 32-bit word; rows 32 apart in an atom are 4 bytes apart).
+
+def _sf(M, nkb, seed=0):
+    rng = np.random.default_rng(seed)
+    return rng.integers(1, 256, size=(M, nkb), dtype=np.uint8)      # never 0
+
+
+@pytest.mark.parametrize("M,nkb", [(128, 4), (256, 8), (384, 16), (130, 4), (1, 8), (1000, 12)])
+def test_swizzle_round_trip_and_padding(M, nkb):
+    sf = _sf(M, nkb, M + nkb)
+    buf = oracle.swizzle_scales(sf)
+    m_pad = -(-M // 128) * 128
+    assert buf.size == m_pad * nkb                      # one byte per (padded row, block)
+    assert np.array_equal(oracle.unswizzle_scales(buf, M, nkb * 16), sf)
+    assert np.count_nonzero(buf) == M * nkb            # padding rows are zero, nothing collides
+
+
+def test_swizzle_is_a_bijection_on_full_atoms():
+    M, nkb = 256, 8
+    r = np.arange(M)[:, None]
+    c = np.arange(nkb)[None, :]
+    # position of (r, c) found by swizzling a one-hot byte per row chunk
+    seen = np.zeros(M * nkb, np.int32)
+    for rr in range(M):
+        for cc in range(nkb):
+            one = np.zeros((M, nkb), np.uint8)
+            one[rr, cc] = 1
+            seen += oracle.swizzle_scales(one).astype(np.int32)
+    assert np.all(seen == 1)
+
+
+def test_swizzle_word_and_quadrant_structure():
+    M, nkb = 128, 8
+    sf = np.zeros((M, nkb), np.uint8)
+    # row 5, blocks 4..7 -> four consecutive bytes (one 32-bit word)
+    sf[5, 4:8] = [11, 12, 13, 14]
+    buf = oracle.swizzle_scales(sf)
+    pos = np.nonzero(buf)[0]
+    assert np.array_equal(buf[pos], [11, 12, 13, 14]) and np.array_equal(np.diff(pos), [1, 1, 1])
+    assert pos[0] % 4 == 0
+    # rows r and r + 32 of an atom, same block: 4 bytes apart
+    sf2 = np.zeros((M, nkb), np.uint8)
+    sf2[7, 1] = 1
+    sf2[39, 1] = 2
+    b2 = oracle.swizzle_scales(sf2)
+    assert np.nonzero(b2 == 2)[0][0] - np.nonzero(b2 == 1)[0][0] == 4
