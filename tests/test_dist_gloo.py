@@ -59,3 +59,35 @@ def test_two_rank_max_timing_and_independent_replicas():
 def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(3.5, torch.device("cpu")) == 3.5
+
+
+def _ref_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank),
+                      LOCAL_RANK=str(rank))
+    import argparse
+    import bench
+    try:
+        args = argparse.Namespace(workload="moe_t512_e8", steps=1, warmup=0, seed=0, gpus=world)
+        out = bench.run_reference(args)
+        q.put((rank, None if out is None else (out["impl"], out["n_gpus"], out["cpu_baseline"]["kind"])))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under torchrun the oracle arm runs on rank 0 alone; other ranks exit
+    without work."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ref_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=300) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert results[1] is None
+    assert results[0] == ("reference", world, "oracle")
