@@ -30,6 +30,9 @@ def _p(t):
 
 
 def _stream(device=None):
+    if device is not None and torch.device(device).type != "cuda":
+        raise ValueError(f"the NVFP4 kernels run on CUDA tensors only (got a tensor on {device}); "
+                         "there is no CPU path")
     return torch.cuda.current_stream(device).cuda_stream
 
 

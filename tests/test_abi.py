@@ -107,3 +107,12 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         _lib.load()
+
+
+def test_api_rejects_non_cuda_tensors():
+    """The binding has no CPU path: host tensors are refused with a clear error."""
+    import torch
+    from quantization_nvfp4_quantize_b200 import api
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        api.quantize(x)
