@@ -10,16 +10,19 @@ Element-wise and block-wise quantization arithmetic lives in plain C
 this module adds the layout transforms and the dense algebra (routing glue,
 matrix products in binary64, SiLU) on numpy.  Every function cites the passage
 of the QUADS pages it follows; readings of what the pages leave open are
-marked READING and listed in the design doc.
+marked READING.
 
 Pins (tests/test_oracle_*.py): exhaustive nearest-value checks of the E2M1 and
-E4M3 encoders, the format tables in tests/golden/, closed forms (block maximum
-maps to +-6, |R| <= d, all-zero tensors), selection against a full sort,
-routing against a sort-based top-k, and the matrix products against brute
-force loops on tiny shapes plus special-case reductions.
-
-Parity unpinned: the scale-factor byte layout (``swizzle_scales``) has no pin
-on the CPU; it is pinned on the GPU by the tensor-core GEMM matching the
+E4M3 encoders, the format tables in tests/golden/, an exact rational
+re-derivation of the block arithmetic (including stored cases where a
+reciprocal-multiply or double-rounded variant would give other codes),
+closed forms (block maximum maps to +-6, |R| <= d, all-zero tensors),
+selection against a full sort, routing against a sort-based top-k, the
+matrix products against brute force loops on tiny shapes plus special-case
+reductions, and structural pins of the scale-factor byte layout (a bijection
+onto the padded buffer with an exact inverse, zero padding rows, one 32-bit
+word per row and 64-element group).  The exact byte positions of that layout
+are pinned on the GPU, where the tensor-core GEMM consumes it and matches the
 brute-force dense product.
 """
 from __future__ import annotations
@@ -187,16 +190,16 @@ def quantize(x: np.ndarray, s_t: float | None = None) -> Quantized:
 
 
 def dequantize(codes: np.ndarray, sf: np.ndarray, s_t: float) -> np.ndarray:
-    """xhat = fl(e2m1(q) * fl(sf * s_t)) in binary32 from packed codes and
-    row-major scale codes."""
+    """xhat = fl(e2m1(q) * sf * s_t) in binary32 from packed codes and
+    row-major scale codes (e2m1 * sf is exact, so one rounding)."""
     M = codes.shape[0]
     K = codes.shape[1] * 2
     q = np.empty((M, K), np.uint8)
     q[:, 0::2] = codes & 0xF
     q[:, 1::2] = codes >> 4
-    d = (e4m3_decode(sf).astype(np.float32) * np.float32(s_t)).astype(np.float32)
-    d = np.repeat(d, 16, axis=1)
-    return (e2m1_decode(q).astype(np.float32) * d).astype(np.float32)
+    sfv = np.repeat(e4m3_decode(sf).astype(np.float32), 16, axis=1)
+    qsf = (e2m1_decode(q).astype(np.float32) * sfv).astype(np.float32)
+    return (qsf * np.float32(s_t)).astype(np.float32)
 
 
 def swizzle_scales(sf: np.ndarray, m_pad: int | None = None) -> np.ndarray:

@@ -155,40 +155,43 @@ float oracle_tensor_scale_from_amax(float A)
 /* ------------------------------------------------------ block quantization */
 
 /* One 16-element block (see the header comment of oracle_quantize for the
- * steps).  Writes 16 element codes, returns the E4M3 scale code. */
-static uint8_t quantize_block(const float xb[16], float s_t, uint8_t q[16], float *d_out)
+ * steps).  Writes 16 element codes and their dequantized values, returns the
+ * E4M3 scale code. */
+static uint8_t quantize_block(const float xb[16], float s_t, uint8_t q[16], float xh[16])
 {
     float amax_b = 0.0f;
     for (int i = 0; i < 16; ++i) {
         float a = fabsf(xb[i]);
         if (a > amax_b) amax_b = a;
     }
-    float e6 = 6.0f * s_t;
-    float r6 = 1.0f / e6;
-    float v = amax_b * r6;                          /* ~ amax_b / (6 s_t) */
+    float v = (amax_b / 6.0f) / s_t;                /* amax/6, in units of s_t */
     uint8_t sf_code = oracle_e4m3_encode(v);
     float sf = (float)oracle_e4m3_decode(sf_code);
-    float d = sf * s_t;                             /* block dequant scale */
-    float rcp = (d == 0.0f) ? 0.0f : 1.0f / d;
+    float d = sf * s_t;                             /* the block's scale */
     for (int i = 0; i < 16; ++i) {
-        float y = xb[i] * rcp;
+        /* a zero scale (only when the block is negligible next to the tensor
+         * maximum) maps every element to a signed zero */
+        float y = (d == 0.0f) ? xb[i] * 0.0f : xb[i] / d;
         q[i] = oracle_e2m1_encode(y);
+        float qsf = (float)oracle_e2m1_decode(q[i]) * sf;   /* exact: 2 x 4 significant bits */
+        xh[i] = qsf * s_t;
     }
-    *d_out = d;
     return sf_code;
 }
 
 /*
  * NVFP4 quantization of a row-major bf16 matrix X [M x K] (K % 16 == 0) with
  * a given per-tensor scale s_t.  For each 16-element block along K:
- *   1. a_b = max |x|;  v = a_b * fl(1 / fl(6 * s_t));
+ *   1. a_b = max |x|;  v = fl(fl(a_b / 6) / s_t): the block maximum over the
+ *      largest E2M1 magnitude, in units of the tensor scale;
  *   2. sf = E4M3(v) (nearest even, saturating);  d = fl(sf * s_t);
- *   3. q_i = E2M1(fl(x_i * fl(1/d)))  (all codes +-0 when d == 0);
- *   4. xhat_i = fl(e2m1(q_i) * d);  R_i = fl(x_i - xhat_i).
- * READING: the pages describe the format only by name; the reciprocal-multiply
- * form (one correctly rounded reciprocal per block) and d = fl(sf * s_t) used
- * for both quantize and dequantize are this build's reading, identical on
- * both sides.
+ *   3. q_i = E2M1(fl(x_i / d))  (all codes +-0 when d == 0);
+ *   4. xhat_i = fl(e2m1(q_i) * sf * s_t), the dequantized value (the product
+ *      e2m1 * sf is exact, so this is one rounding of the exact triple
+ *      product);  R_i = fl(x_i - xhat_i).
+ * READING: the pages name the format but not its arithmetic; every step is
+ * the plain binary32 evaluation of its definition, left to right, one
+ * rounding per operation.
  * Outputs (any may be NULL):
  *   codes  [M x K/2]  element 2j in bits 0..3, element 2j+1 in bits 4..7
  *   sf     [M x K/16] E4M3 scale codes, plain row-major (not swizzled)
@@ -202,20 +205,18 @@ void oracle_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, float
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < M; ++r) {
         for (int64_t b = 0; b < nkb; ++b) {
-            float xb[16];
+            float xb[16], xh[16];
             uint8_t q[16];
-            float d;
             for (int i = 0; i < 16; ++i)
                 xb[i] = oracle_bf16_to_f32(x[r * ldx + b * 16 + i]);
-            uint8_t sc = quantize_block(xb, s_t, q, &d);
+            uint8_t sc = quantize_block(xb, s_t, q, xh);
             if (sf) sf[r * nkb + b] = sc;
             if (codes)
                 for (int i = 0; i < 8; ++i)
                     codes[r * (K / 2) + b * 8 + i] = (uint8_t)(q[2 * i] | (q[2 * i + 1] << 4));
             for (int i = 0; i < 16; ++i) {
-                float xh = (float)oracle_e2m1_decode(q[i]) * d;
-                if (xhat) xhat[r * K + b * 16 + i] = xh;
-                if (resid) resid[r * K + b * 16 + i] = xb[i] - xh;
+                if (xhat) xhat[r * K + b * 16 + i] = xh[i];
+                if (resid) resid[r * K + b * 16 + i] = xb[i] - xh[i];
             }
         }
     }

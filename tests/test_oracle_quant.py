@@ -65,8 +65,9 @@ def test_block_max_maps_to_six_and_residual_bound():
     assert np.all((qmax[normal] & 7) == 7), "block maximum must map to magnitude 6"
     R = qz.resid.reshape(256, 32, 16).astype(np.float64)
     assert np.all(np.abs(R) <= d[..., None].astype(np.float64) * (1 + 2.0 ** -20))
-    # xhat = e2m1 * d exactly as stated
-    xh = (oracle.e2m1_decode(q).astype(np.float32) * d[..., None]).astype(np.float32)
+    # xhat = fl(e2m1 * sf * s_t), one rounding of the exact product
+    qsf = (oracle.e2m1_decode(q) * sf[..., None]).astype(np.float32)
+    xh = (qsf * np.float32(qz.s_t)).astype(np.float32)
     assert np.array_equal(xh.reshape(256, 512), qz.xhat)
     assert np.array_equal((xf - xh).reshape(256, 512), qz.resid)
 
