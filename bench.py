@@ -39,14 +39,15 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP4_PER_BF16 = 4.0          # nominal dense FP4 : BF16 tensor-core ratio (9 : 2.25 PFLOP/s)
+NOMINAL_FP4_TFLOPS = 9000.0  # B200 dense FP4, datasheet (context)
 QUANT_BYTES_PER_ELEM = 2.5625   # 2 B bf16 read + 0.5 B codes + 1/16 B scale written
 
 # DRAM traffic of k_moe_gemm per launch (dram__bytes_read.sum + dram__bytes_write.sum,
-# averaged over the gate/up and down launches of one step) from the ncu capture
-# summarised in profiles/k_moe_gemm_moe_t16384_e128.md, valid only for the kernel
-# code it was taken on: sha256 of gemm.cu + ptx.cuh + common.cuh with comments
-# removed and whitespace collapsed (a comment edit leaves the kernel, and the
-# figure, as is).
+# averaged over the gate/up and down launches of one step) from a one-pass ncu
+# capture of this benchmark's two timed steps (the ncu command is kept with the
+# profile summaries), valid only for the kernel code it was taken on: sha256 of
+# gemm.cu + ptx.cuh + common.cuh with comments removed and whitespace collapsed
+# (a comment edit leaves the kernel, and the figure, as is).
 GEMM_TRAFFIC = {"bytes_per_launch": 2402440832, "sources_sha256": "620d862eca54259eefb401c1710b09ed01b8f62a011824243bf4e7ada3bb76c6"}
 
 
@@ -97,6 +98,7 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-w4a16", action="store_true", help="skip the trainer-side W4A16 line of the default run")
     return ap.parse_args()
 
 
@@ -108,6 +110,19 @@ def peaks():
                     bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), source="measured")
     except Exception:
         return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sus=1400.0, source="fallback")
+
+
+def tensor_peak(p, clk, per_bf16=1.0):
+    """Tensor-core peak for a kernel timed inside the run: the burst bf16
+    figure (a cuBLAS GEMM timed alone at full clock) times the dtype's nominal
+    ratio to bf16, scaled by the median SM clock sampled during the timed
+    region over its maximum (a clock-bound pipe).  Returns (peak, source)."""
+    base = p["bf16"] * per_bf16
+    if clk and clk.get("sm_mhz") and clk.get("sm_max_mhz"):
+        f = min(1.0, float(clk["sm_mhz"]) / float(clk["sm_max_mhz"]))
+        return base * f, (f"{p['source']} bf16 burst x{per_bf16:g} x sampled SM clock "
+                          f"{clk['sm_mhz']:.0f}/{clk['sm_max_mhz']:.0f} MHz")
+    return base, f"{p['source']} bf16 burst x{per_bf16:g} (no clock samples)"
 
 
 def dist_env():
@@ -269,13 +284,16 @@ def run_ours(args):
     M = cfg.tokens * cfg.topk
     quant_elems = cfg.tokens * cfg.hidden + M * cfg.inter
     p = peaks()
-    fp4_peak = p["bf16_sus"] * FP4_PER_BF16
+    fp4_peak, peak_source = tensor_peak(p, clk, FP4_PER_BF16)
     gemm_fp4_tflops = fl["fp4"] * args.steps / (gemm_ms * 1e-3) / 1e12
     gemm_all_tflops = step_flops * args.steps / (gemm_ms * 1e-3) / 1e12
     quant_gbs = quant_elems * QUANT_BYTES_PER_ELEM * args.steps / (quant_ms * 1e-3) / 1e9
 
     # end to end through the public API with host buffers
     e2e = run_e2e(layer, x, logits, args, dev)
+    # the streaming quantize kernel alone (tensor scale given: no amax pass, no
+    # selection or residual), on the layer's own X and h
+    qk = time_quantize_kernel(layer, x, args.steps, dev)
     # per step: route 3, X quantize 5 (amax, quantize, score reduce, select, residual),
     # gather 1, GEMM 1, h quantize 4 (its amax comes from the GEMM epilogue), gather 1, GEMM 1
     n_launch_per_step = 16
@@ -294,16 +312,28 @@ def run_ours(args):
                      "achieved": round(gemm_fp4_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_fp4_tflops / fp4_peak, 4), "traffic": gemm_traffic(),
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
-                     "peak_source": f"{p['source']} bf16 sustained x{FP4_PER_BF16:g} (nominal FP4:BF16)",
+                     "peak_source": peak_source + f" (nominal FP4:BF16 {FP4_PER_BF16:g})",
+                     "frac_nominal_fp4": round(gemm_fp4_tflops / NOMINAL_FP4_TFLOPS, 4),
                      "achieved_incl_rac": round(gemm_all_tflops, 1),
                      "gemm_ms_per_step": round(gemm_ms / args.steps, 4), "launches_per_step": n_gemm // args.steps},
         "quantize": {"gbs": round(quant_gbs, 1), "peak_gbs": p["hbm"], "frac": round(quant_gbs / p["hbm"], 4),
                      "ms_per_step": round(quant_ms / args.steps, 4),
-                     "bytes_per_elem": QUANT_BYTES_PER_ELEM, "elems_per_step": quant_elems},
+                     "bytes_per_elem": QUANT_BYTES_PER_ELEM, "elems_per_step": quant_elems,
+                     "scope": "whole nvfp4_quantize calls (amax, quantize, score reduce, select, RAC residual)",
+                     "kernel": qk},
         "e2e": e2e,
         "gpu_launches": n_launch_per_step * args.steps,
         "clocks": clk,
     }
+    if not args.no_w4a16:
+        # the trainer-side path (weight QDQ + W4A16 grouped GEMMs) on its own
+        # workload, in the same run
+        del layer, x, logits
+        torch.cuda.empty_cache()
+        w = run_ours_w4a16(args, workload="qat_w4a16_e128", emit=False)
+        out["w4a16"] = {k: w[k] for k in ("metric", "value", "unit", "ms_per_step", "roofline", "qdq", "e2e")}
+        out["w4a16"]["config"] = w["config"]["workload"]
+        out["gpu_launches"] += w["gpu_launches"]
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=64)
     if rank == 0:
@@ -311,11 +341,56 @@ def run_ours(args):
     return out
 
 
+def time_quantize_kernel(layer, x_in, steps, dev):
+    """k_quantize (+ its score reduction) alone on the layer's X (written to
+    its k_r routed rows) and h, with the tensor scales the step computed:
+    algorithmic bytes 2 B read + 0.5625 B written per element, and the bytes
+    the X pass moves with its routed copies."""
+    import torch
+    from quantization_nvfp4_quantize_b200 import api
+    r = layer.routing
+    stream = torch.cuda.current_stream(dev)
+    E, H, I, T, kr = layer.E, layer.H, layer.I, layer.T, layer.k_r
+
+    def xq():
+        api.quantize(x_in, rac_k=0, s_t=layer.xq.s_t, dst_rows=r.dst_row, fanout=kr, m_out=layer.m_pad,
+                     want_score=True, out=layer.xq, workspace=layer.ws_x)
+
+    def hq():
+        api.quantize(layer.h, rac_k=0, s_t=layer.hq.s_t, m_out=layer.m_pad, m_valid=r.offsets[E:],
+                     want_score=True, out=layer.hq, workspace=layer.ws_h)
+
+    for _ in range(2):
+        xq(); hq()
+    n = max(3, steps)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        ev[i][0].record(stream); xq(); ev[i][1].record(stream)
+        ev[i][2].record(stream); hq(); ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    x_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n
+    h_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / n
+    h_rows = int(r.offsets[E].item())
+    x_el, h_el = T * H, h_rows * I
+    p = peaks()
+    gbs = lambda b, ms: b / (ms * 1e-3) / 1e9
+    x_alg, h_alg = x_el * QUANT_BYTES_PER_ELEM, h_el * QUANT_BYTES_PER_ELEM
+    x_moved = x_el * (2.0 + kr * 0.5625)
+    tot = gbs(x_alg + h_alg, x_ms + h_ms)
+    return {"gbs": round(tot, 1), "frac": round(tot / p["hbm"], 4), "ms_per_step": round(x_ms + h_ms, 4),
+            "x_pass": {"us": round(x_ms * 1e3, 1), "gbs": round(gbs(x_alg, x_ms), 1),
+                       "gbs_moved_incl_routed_copies": round(gbs(x_moved, x_ms), 1), "elems": x_el},
+            "h_pass": {"us": round(h_ms * 1e3, 1), "gbs": round(gbs(h_alg, h_ms), 1), "elems": h_el},
+            "bytes_per_elem": QUANT_BYTES_PER_ELEM,
+            "scope": "k_quantize with scores and the score reduction; tensor scale given"}
+
+
 METRIC_W4A16 = "W4A16 BF16 grouped MoE GEMM TFLOPS and % BF16 peak; weight QDQ GB/s and % HBM"
 QDQ_BYTES_PER_ELEM = 4.0    # 2 B bf16 weight read + 2 B bf16 fake-quantized weight written
 
 
-def run_ours_w4a16(args):
+def run_ours_w4a16(args, workload=None, emit=True):
     """Trainer-side step (asymmetric QAT): NVFP4 fake quantization of every
     expert weight (they change every optimizer step), then the W4A16 layer
     forward: routing, routed-row gather of X, BF16 grouped gate/up GEMM with
@@ -329,7 +404,7 @@ def run_ours_w4a16(args):
     assert torch.cuda.is_available(), "bench.py needs a CUDA device"
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    cfg = wl.CONFIGS[args.workload]
+    cfg = wl.CONFIGS[workload or args.workload]
     seed = args.seed + rank
     x = wl.activations(cfg, seed, device=dev)
     logits = wl.router_logits(cfg, seed, device=dev)
@@ -385,7 +460,7 @@ def run_ours_w4a16(args):
     gemm_ms = sum(s_.elapsed_time(e_) for s_, e_ in ev["gemm"])
     qdq_ms = sum(s_.elapsed_time(e_) for s_, e_ in ev["qdq"])
     p = peaks()
-    bf16_peak = p["bf16_sus"]
+    bf16_peak, peak_source = tensor_peak(p, clk, 1.0)
     gemm_tflops = step_flops * args.steps / (gemm_ms * 1e-3) / 1e12
     w_elems = w13.numel() + w2.numel()
     qdq_gbs = w_elems * QDQ_BYTES_PER_ELEM * args.steps / (qdq_ms * 1e-3) / 1e9
@@ -428,7 +503,7 @@ def run_ours_w4a16(args):
         "roofline": {"bound": "tensor", "kernel": "k_moe_gemm (BF16 stages)",
                      "achieved": round(gemm_tflops, 1), "peak": round(bf16_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tflops / bf16_peak, 4), "traffic": None,
-                     "peak_source": f"{p['source']} bf16 sustained",
+                     "peak_source": peak_source,
                      "gemm_ms_per_step": round(gemm_ms / args.steps, 4), "launches_per_step": 2},
         "qdq": {"gbs": round(qdq_gbs, 1), "peak_gbs": p["hbm"], "frac": round(qdq_gbs / p["hbm"], 4),
                 "ms_per_step": round(qdq_ms / args.steps, 4), "bytes_per_elem": QDQ_BYTES_PER_ELEM,
@@ -440,7 +515,7 @@ def run_ours_w4a16(args):
         "gpu_launches": 10 * args.steps,
         "clocks": clk,
     }
-    if rank == 0:
+    if rank == 0 and emit:
         print(json.dumps(out), flush=True)
     return out
 

@@ -45,9 +45,10 @@
  *           (r%32)*16 + ((r%128)/32)*4 + c%4.  Buffer size:
  *           ceil(rows/128)*128 * K/16 bytes.  Rows are padded to 128.
  *   s_t     float32 per tensor: s_t = max|x| / 2688 (1 for an all-zero tensor).
- *   Per 16-block with amax a: sf = E4M3_rne(a * (1/(6 s_t))), d = sf*s_t,
- *   q = E2M1_rne(x * (1/d)), dequantized value xhat = e2m1(q)*d, residual
- *   R = x - xhat (binary32 throughout).
+ *   Per 16-block with amax a (binary32, one rounding per operation):
+ *   sf = E4M3_rne(fl(fl(a/6)/s_t)), d = fl(sf*s_t), q = E2M1_rne(fl(x/d)),
+ *   dequantized value xhat = fl(e2m1(q)*sf*s_t) (e2m1*sf is exact), residual
+ *   R = fl(x - xhat).
  */
 #ifndef NVFP4_QUADS_H
 #define NVFP4_QUADS_H

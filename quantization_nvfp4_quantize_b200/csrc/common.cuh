@@ -115,6 +115,17 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float v)
     return r & 0xFFu;
 }
 
+// Two non-negative floats -> their E4M3 codes: `lo` in bits 0..7, `hi` in 8..15.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b16 t;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u16 %0, t;\n\t}"
+        : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // E4M3 code -> value (exact in f16 and f32).
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code)
 {
@@ -126,55 +137,171 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code)
     return __low2float(*reinterpret_cast<__half2 *>(&h2));
 }
 
+// E4M3 code -> the value in both halves of an f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3_to_h2(uint32_t code)
+{
+    uint32_t h2;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+        : "=r"(h2) : "r"((code & 0xFFu) * 0x101u));
+    return h2;
+}
+
 // Per-tensor scale from the tensor's max |x|: s_t = A / 2688, 1 if A == 0.
 __device__ __forceinline__ float tensor_scale_from_amax(float A)
 {
     return A == 0.0f ? 1.0f : __fdiv_rn(A, 2688.0f);
 }
 
-// Block scale factor pieces shared by every quantizing kernel.
-struct BlockScale {
-    uint32_t sf_code;  // E4M3 code
-    float d;           // block dequantization scale fl(sf * s_t)
-    float rcp;         // fl(1 / d), 0 when d == 0
+// ------------------------------------------------------- NVFP4 block steps
+//
+// Definitions (binary32, one rounding per operation):
+//   block scale   sf = E4M3(fl(fl(a/6) / s_t)), a = max |x| over the block
+//   element code  q  = E2M1(fl(x / d)), d = fl(sf * s_t)
+//   dequantized   xhat = fl(e2m1(q) * sf * s_t)   (e2m1 * sf is exact)
+//   residual      R = fl(x - xhat)
+//
+// Both encodings are monotone in their (real) argument, so a decision can be
+// taken from two multiplications that bracket the exact quotient: with
+// lo = fl(fl(1/den) * (1 - 2^-20)) and hi = fl(fl(1/den) * (1 + 2^-20)),
+//   num * lo < num / den * (1 - 2^-21) and num * hi > num / den * (1 + 2^-21),
+// which encloses every value within a few binary32 roundings of num / den
+// (a rounded reciprocal and product move a value by at most 2^-23 relative;
+// fl(fl(a/6) / s_t) by at most 2^-23 from a / (6 s_t)).  Rounding to binary32
+// is monotone, so fl(num * lo) <= fl(num / den) <= fl(num * hi); when the two
+// brackets encode to the same code, that is the code of the exact-division
+// definition.  Otherwise (an argument within about 2^-20 of a rounding
+// boundary: a few per million elements) the IEEE divisions are evaluated.
+
+// Bracketing multipliers (lo, hi) around 1/den.
+__device__ __forceinline__ float2 recip_bracket(float den)
+{
+    const float r = __frcp_rn(den);
+    return make_float2(__fmul_rn(r, 1.0f - 0x1p-20f), __fmul_rn(r, 1.0f + 0x1p-20f));
+}
+
+// E4M3 code of the block scale fl(fl(a/6) / s_t), a >= 0; r6 = bracket of
+// 1/(6 s_t) (recip_bracket(fl(6 s_t)) encloses it: fl(6 s_t) is within 2^-24).
+__device__ __forceinline__ uint32_t block_scale_code(float a, float s_t, float2 r6)
+{
+    const uint32_t c2 = cvt_e4m3x2(__fmul_rn(a, r6.x), __fmul_rn(a, r6.y));
+    const uint32_t c = c2 & 0xFFu;
+    if ((c2 >> 8) == c) return c;
+    return cvt_e4m3(__fdiv_rn(__fdiv_rn(a, 6.0f), s_t));
+}
+
+// Per E4M3 scale code, the per-tensor quantities of a block: its scale
+// d = fl(sf * s_t), the bracket of 1/d (both 0 when d == 0: every element
+// then maps to a signed zero), and sf in both halves of an f16x2.
+struct BlockConst {
+    float d, rlo, rhi;
+    uint32_t sf_h2;
 };
 
-__device__ __forceinline__ BlockScale block_scale(float amax_b, float s_t, float r6)
+__device__ __forceinline__ BlockConst block_const(uint32_t code, float s_t)
 {
-    BlockScale b;
-    b.sf_code = cvt_e4m3(__fmul_rn(amax_b, r6));
-    float sf = e4m3_to_f32(b.sf_code);
-    b.d = __fmul_rn(sf, s_t);
-    b.rcp = (b.d == 0.0f) ? 0.0f : __frcp_rn(b.d);
+    BlockConst b;
+    b.d = __fmul_rn(e4m3_to_f32(code), s_t);
+    if (b.d == 0.0f) {
+        b.rlo = b.rhi = 0.0f;
+    } else {
+        const float2 r = recip_bracket(b.d);
+        b.rlo = r.x;
+        b.rhi = r.y;
+    }
+    b.sf_h2 = e4m3_to_h2(code);
     return b;
 }
 
-// r6 = fl(1 / fl(6 * s_t)), the per-tensor factor mapping a block max to its
-// E4M3 scale value.
-__device__ __forceinline__ float block_r6(float s_t) { return __frcp_rn(__fmul_rn(6.0f, s_t)); }
-
-// Quantize 8 consecutive elements (one lane's half of a 16-block whose other
-// half is held by lane ^ 1) given the block scale.  Returns 4 code bytes
-// (little-endian element order) and the dequantized values.
-__device__ __forceinline__ uint32_t quant8(const float v[8], const BlockScale &b, float xh[8])
+// Packed binary32 pairs (sm_100a f32x2 arithmetic, round to nearest even).
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
 {
-    float y[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(v[i], b.rcp);
-    uint32_t w = cvt_e2m1x8(y);
-    float q[8];
-    e2m1x8_to_f32(w, q);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) xh[i] = __fmul_rn(q[i], b.d);
-    return w;
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
 }
 
-// Dequantized value of a single element given its block scale.
-__device__ __forceinline__ float quant1_xhat(float v, const BlockScale &b)
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
 {
-    uint32_t byte = cvt_e2m1x2(__fmul_rn(v, b.rcp), 0.0f);
-    float2 q = e2m1x2_to_f32(byte);
-    return __fmul_rn(q.x, b.d);
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+        "fma.rn.f32x2 d, a, b, c;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// One bf16x2 word -> its two values as a float pair (exact): .x = low half.
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w)
+{
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// E2M1 codes of 8 elements (one lane's half of a 16-block; 4 bytes, element
+// 2i in the low nibble of byte i) given the block's constants.
+__device__ __forceinline__ uint32_t element_codes8(const float2 v[4], const BlockConst &b)
+{
+    float ylo[8], yhi[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 lo = mul2(v[i], make_float2(b.rlo, b.rlo));
+        const float2 hi = mul2(v[i], make_float2(b.rhi, b.rhi));
+        ylo[2 * i] = lo.x; ylo[2 * i + 1] = lo.y;
+        yhi[2 * i] = hi.x; yhi[2 * i + 1] = hi.y;
+    }
+    const uint32_t wlo = cvt_e2m1x8(ylo);
+    if (wlo == cvt_e2m1x8(yhi)) return wlo;
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        y[2 * i] = __fdiv_rn(v[i].x, b.d);
+        y[2 * i + 1] = __fdiv_rn(v[i].y, b.d);
+    }
+    return cvt_e2m1x8(y);
+}
+
+// Dequantized values of 8 elements from their codes: pairs
+// xhat = fl(fl(e2m1 * sf) * s_t), the e2m1 * sf products exact in f16.  The
+// final multiply is scalar mul.rn.f32: the code generator fuses a packed
+// f32x2 multiply with a following packed subtraction into one fused
+// multiply-add, which would skip the rounding of xhat the residual depends on.
+__device__ __forceinline__ void dequant8(uint32_t w, uint32_t sf_h2, float s_t, float2 xh[4])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t q2;
+        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+            "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+            : "=r"(q2) : "r"(w >> (8 * i)));
+        uint32_t p2;
+        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p2) : "r"(q2), "r"(sf_h2));
+        const float2 qsf = __half22float2(*reinterpret_cast<__half2 *>(&p2));
+        xh[i] = make_float2(__fmul_rn(qsf.x, s_t), __fmul_rn(qsf.y, s_t));
+    }
+}
+
+// Residuals R = fl(x - xhat) of 8 elements (scalar sub.rn.f32, see dequant8).
+__device__ __forceinline__ void residual8(const float2 v[4], const float2 xh[4], float2 R[4])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) R[i] = make_float2(__fsub_rn(v[i].x, xh[i].x), __fsub_rn(v[i].y, xh[i].y));
+}
+
+// Dequantized value fl(fl(e2m1(q) * sf) * s_t) of a single element.
+__device__ __forceinline__ float element_xhat1(float v, const BlockConst &b, float s_t)
+{
+    const uint32_t c2 = cvt_e2m1x2(__fmul_rn(v, b.rlo), __fmul_rn(v, b.rhi));
+    uint32_t q = c2 & 15u;
+    if ((c2 >> 4) != q) q = cvt_e2m1x2(__fdiv_rn(v, b.d), 0.0f) & 15u;
+    const float sf = __low2float(*reinterpret_cast<const __half2 *>(&b.sf_h2));
+    return __fmul_rn(__fmul_rn(e2m1x2_to_f32(q).x, sf), s_t);
 }
 
 // Status word helpers.

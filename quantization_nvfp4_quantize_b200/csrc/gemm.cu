@@ -614,16 +614,17 @@ static nvfp4_status launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, con
                            const CUtensorMap &tm_rb, const CUtensorMap &tm_sfa, const CUtensorMap &tm_sfb,
                            const Params &p, int units, cudaStream_t st)
 {
-    static bool attr_done[64];
+    static std::once_flag once[64];
+    static cudaError_t attr_err[64];
     auto kern = k_moe_gemm<STAGES, PAIR, STAGING>;
     const uint32_t smem = Cfg<STAGES, PAIR, STAGING>::SMEM;
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return check_launch("moe_w4a4_grouped_gemm_rac: smem attribute");
-        attr_done[dev] = true;
-    }
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return check_launch("k_moe_gemm: device");
+    std::call_once(once[dev], [&] {
+        attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
+    if (attr_err[dev] != cudaSuccess)
+        return set_error(NVFP4_ERR_CUDA, "k_moe_gemm: smem attribute: %s", cudaGetErrorString(attr_err[dev]));
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     cfg.gridDim = dim3((unsigned)(PAIR ? 2 * units : units));

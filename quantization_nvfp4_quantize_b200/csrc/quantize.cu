@@ -36,6 +36,17 @@ constexpr uint32_t QSMEM = QSTAGES * QROWS * QCHUNK * 2;   // 64 KB of tiles per
 
 // -------------------------------------------------------------------- amax
 
+// max |x| per group.  |bf16| bit patterns order like their values, so the
+// maximum is taken on pairs of 16-bit integers; every thread keeps 4
+// independent 16-byte loads in flight.  Contiguous tensors (ldx == K) are
+// swept as one flat array; otherwise warps take whole rows.
+__device__ __forceinline__ uint32_t absmax_pairs(uint32_t m2, uint4 u)
+{
+    const uint32_t a = __vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu);
+    const uint32_t b = __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu);
+    return __vmaxu2(m2, __vmaxu2(a, b));
+}
+
 __global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16 *__restrict__ x, int64_t ldx,
                                               int64_t M, int64_t K, const int32_t *__restrict__ m_valid,
                                               int64_t group_stride, unsigned int *__restrict__ amax_bits)
@@ -43,22 +54,28 @@ __global__ void __launch_bounds__(256) k_amax(const __nv_bfloat16 *__restrict__ 
     int64_t Me = M;
     if (m_valid) Me = min(Me, (int64_t)max(*m_valid, 0));
     const __nv_bfloat16 *xg = x + (int64_t)blockIdx.y * group_stride;
-    const int vec_per_row = (int)(K / 8);
-    float m = 0.0f;
-    // each warp sweeps whole rows; rows are strided over all warps of the grid
-    const int lane = threadIdx.x & 31;
-    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t r = gw; r < Me; r += nw) {
-        const uint4 *row = reinterpret_cast<const uint4 *>(xg + r * ldx);
-        for (int v = lane; v < vec_per_row; v += 32) {
-            uint4 u = __ldg(row + v);
-            m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(u.x)), fabsf(bf16hi(u.x))),
-                               fmaxf(fabsf(bf16lo(u.y)), fabsf(bf16hi(u.y)))));
-            m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(u.z)), fabsf(bf16hi(u.z))),
-                               fmaxf(fabsf(bf16lo(u.w)), fabsf(bf16hi(u.w)))));
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    uint32_t m2 = 0u;
+    if (ldx == K) {
+        const uint4 *v = reinterpret_cast<const uint4 *>(xg);
+        const int64_t total = Me * (K / 8);
+        int64_t i = tid;
+        for (; i + 3 * nthr < total; i += 4 * nthr) {
+            const uint4 u0 = __ldg(v + i), u1 = __ldg(v + i + nthr), u2 = __ldg(v + i + 2 * nthr),
+                        u3 = __ldg(v + i + 3 * nthr);
+            m2 = absmax_pairs(absmax_pairs(absmax_pairs(absmax_pairs(m2, u0), u1), u2), u3);
+        }
+        for (; i < total; i += nthr) m2 = absmax_pairs(m2, __ldg(v + i));
+    } else {
+        const int lane = threadIdx.x & 31;
+        const int vpr = (int)(K / 8);
+        for (int64_t r = tid >> 5; r < Me; r += nthr >> 5) {
+            const uint4 *row = reinterpret_cast<const uint4 *>(xg + r * ldx);
+            for (int j = lane; j < vpr; j += 32) m2 = absmax_pairs(m2, __ldg(row + j));
         }
     }
+    float m = fmaxf(bf16lo(m2), bf16hi(m2));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     __shared__ float wm[8];
@@ -114,17 +131,28 @@ __device__ __forceinline__ bool qwait(uint32_t bar, uint32_t parity, volatile in
     }
 }
 
+constexpr int QFAN_SLOTS = 4;         // per-warp ring of staged code rows for the fan-out bulk stores
+
 // One CTA = 8 warps on one 256-channel column chunk and one range of rows.
 // Thread 0 streams 32-row x 256-channel bf16 tiles (16 KB) through a 4-stage
 // shared-memory ring with TMA; warp w quantizes tile rows w, w+8, w+16, w+24,
-// each lane 8 channels (a lane pair is one 16-element block).
-template <bool SCORE>
+// each lane 8 channels (a lane pair is one 16-element block).  Arithmetic on
+// element pairs uses the packed f32x2 instructions.
+//   SCORE  accumulate the channels' residual sums of squares
+//   QDQ    write bf16(xhat) (weight fake quantization)
+// With dst_rows, the codes of a row (128 contiguous bytes per warp) are staged
+// in shared memory and written to each destination row by one bulk copy per
+// destination; the scale words go out as 4-byte stores, one per lane.
+template <bool SCORE, bool QDQ>
 __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __grid_constant__ CUtensorMap tm_x,
                                                                      QuantParams p)
 {
     extern __shared__ __align__(128) uint8_t qsm[];              // QSTAGES x QROWS x box_inner bf16
     __shared__ uint64_t full_bar[QSTAGES], empty_bar[QSTAGES];
     __shared__ int abort_sm;
+    __shared__ float4 btab[128];                                  // per E4M3 code: d, rlo, rhi, sf_h2
+    __shared__ int32_t fdst[QTHREADS / 32][QROWS / (QTHREADS / 32)][32];      // fan-out rows of a warp's 4 rows
+    __shared__ __align__(128) uint32_t fstage[QTHREADS / 32][QFAN_SLOTS][32]; // staged code rows
     volatile int *abort_flag = &abort_sm;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -136,9 +164,9 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
     const uint32_t pitch = (uint32_t)p.box_inner * 2u;            // bytes per tile row in shared memory
     const uint32_t tile_bytes = pitch * QROWS;
 
-    float s_t = p.s_t_in ? p.s_t_in[g] : tensor_scale_from_amax(__uint_as_float(p.amax_bits[g]));
+    const float s_t = p.s_t_in ? p.s_t_in[g] : tensor_scale_from_amax(__uint_as_float(p.amax_bits[g]));
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.s_t_out) p.s_t_out[g] = s_t;
-    const float r6 = block_r6(s_t);
+    const float2 r6 = recip_bracket(__fmul_rn(6.0f, s_t));
 
     int64_t Me = p.M;
     if (p.m_valid) Me = min(Me, (int64_t)max(*p.m_valid, 0));
@@ -149,16 +177,14 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
 
     uint8_t *codes = p.codes ? p.codes + g * p.codes_gstride : nullptr;
     uint8_t *scales = p.scales ? p.scales + g * p.scales_gstride : nullptr;
-    __nv_bfloat16 *qdq = p.qdq ? p.qdq + g * p.qdq_gstride : nullptr;
+    __nv_bfloat16 *qdq = QDQ ? p.qdq + g * p.qdq_gstride : nullptr;
+    const int fanout = p.dst_rows ? p.fanout : 0;
 
-    // E4M3 code -> (d, 1/d) = (fl(sf * s_t), fl(1 / d)): a block scale takes at
-    // most 127 values per tensor, so each is computed once here rather than
-    // once per block (same arithmetic, same values).
-    __shared__ float2 dtab[128];
-    __shared__ longlong2 fan[QTHREADS / 32][32];                 // per-warp fan-out offsets of one row
+    // E4M3 code -> the block's constants: a block scale takes at most 127
+    // values per tensor, so each is computed once here rather than per block.
     if (threadIdx.x < 128) {
-        const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), s_t);
-        dtab[threadIdx.x] = make_float2(d, d == 0.0f ? 0.0f : __frcp_rn(d));
+        const BlockConst b = block_const(threadIdx.x, s_t);
+        btab[threadIdx.x] = make_float4(b.d, b.rlo, b.rhi, __uint_as_float(b.sf_h2));
     }
     if (threadIdx.x == 0) {
         for (int st = 0; st < QSTAGES; ++st) {
@@ -181,12 +207,16 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
         }
     }
 
-    float acc32[8];
+    float2 acc32[4];
     double acc64[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) { acc32[i] = 0.0f; acc64[i] = 0.0; }
+    for (int i = 0; i < 4; ++i) acc32[i] = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc64[i] = 0.0;
 
-    const int64_t kb0 = c >> 4;                 // first block of the 4-block group (lanes 8j)
+    const int64_t kb0 = c >> 4;                 // first block of the lane octet's 4-block group (lanes 8j)
+    const uint32_t code_bytes = (uint32_t)(min((int64_t)QCHUNK, K - c0) / 2);   // one row's codes in this chunk
+    int fan_slot = 0;
     int it = 0;
     for (; it < n_iter; ++it) {
         const int st = it % QSTAGES;
@@ -195,86 +225,93 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
         if (lane == 0) ok = qwait(ptx::smem_u32(&full_bar[st]), ph, abort_flag, p.dev_status);
         if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
         const uint8_t *tile = qsm + st * tile_bytes;
+        const int64_t rt = r0 + (int64_t)it * QROWS;             // first row of the tile
+        if (fanout) {
+            // this warp's 4 rows x fanout destinations, fetched once per tile
+            for (int e = lane; e < (QROWS / (QTHREADS / 32)) * fanout; e += 32) {
+                const int i = e / fanout, j = e - i * fanout;
+                const int64_t r = rt + warp + i * (QTHREADS / 32);
+                fdst[warp][i][j] = r < r1 ? p.dst_rows[r * fanout + j] : -1;
+            }
+            __syncwarp();
+        }
 #pragma unroll
         for (int i = 0; i < QROWS / (QTHREADS / 32); ++i) {
             const int lr = warp + i * (QTHREADS / 32);            // row inside the tile
-            const int64_t r = r0 + (int64_t)it * QROWS + lr;
+            const int64_t r = rt + lr;
             if (r >= r1) break;                                   // warp-uniform
-            uint4 u = active ? *reinterpret_cast<const uint4 *>(tile + lr * pitch + lane * 16)
-                             : make_uint4(0u, 0u, 0u, 0u);
-            float v[8];
-            v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-            v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
-            float m = fabsf(v[0]);
-#pragma unroll
-            for (int k = 1; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
+            const uint4 u = active ? *reinterpret_cast<const uint4 *>(tile + lr * pitch + lane * 16)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            float2 v[4] = {bf16x2_to_f2(u.x), bf16x2_to_f2(u.y), bf16x2_to_f2(u.z), bf16x2_to_f2(u.w)};
+            float m = fmaxf(fmaxf(fmaxf(fabsf(v[0].x), fabsf(v[0].y)), fmaxf(fabsf(v[1].x), fabsf(v[1].y))),
+                            fmaxf(fmaxf(fabsf(v[2].x), fabsf(v[2].y)), fmaxf(fabsf(v[3].x), fabsf(v[3].y))));
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            BlockScale bs;
-            bs.sf_code = cvt_e4m3(__fmul_rn(m, r6));
-            {
-                const float2 dr = dtab[bs.sf_code];
-                bs.d = dr.x;
-                bs.rcp = dr.y;
-            }
-            float xh[8];
-            uint32_t cw = quant8(v, bs, xh);
-
-            // gather the 4 scale codes of blocks kb0..kb0+3 onto lanes 8j
-            uint32_t s1 = __shfl_down_sync(0xffffffffu, bs.sf_code, 2);
-            uint32_t s2 = __shfl_down_sync(0xffffffffu, bs.sf_code, 4);
-            uint32_t s3 = __shfl_down_sync(0xffffffffu, bs.sf_code, 6);
-            uint32_t sw = bs.sf_code | (s1 << 8) | (s2 << 16) | (s3 << 24);
-
-            if (active) {
+            const uint32_t sf_code = block_scale_code(m, s_t, r6);
+            const float4 bt = btab[sf_code];
+            const BlockConst b{bt.x, bt.y, bt.z, __float_as_uint(bt.w)};
+            const uint32_t cw = element_codes8(v, b);
+            if (SCORE || QDQ) {
+                float2 xh[4];
+                dequant8(cw, b.sf_h2, s_t, xh);
                 if (SCORE) {
+                    float2 R[4];
+                    residual8(v, xh, R);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        float R = __fsub_rn(v[k], xh[k]);
-                        acc32[k] = fmaf(R, R, acc32[k]);
-                    }
+                    for (int k = 0; k < 4; ++k) acc32[k] = fma2(R[k], R[k], acc32[k]);
                 }
-                if (qdq) {
+                if (QDQ && active) {
                     uint4 o;
-                    o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[0])) |
-                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[1])) << 16);
-                    o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[2])) |
-                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[3])) << 16);
-                    o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[4])) |
-                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[5])) << 16);
-                    o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[6])) |
-                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(xh[7])) << 16);
+                    __nv_bfloat162 h;
+                    h = __floats2bfloat162_rn(xh[0].x, xh[0].y); o.x = *reinterpret_cast<uint32_t *>(&h);
+                    h = __floats2bfloat162_rn(xh[1].x, xh[1].y); o.y = *reinterpret_cast<uint32_t *>(&h);
+                    h = __floats2bfloat162_rn(xh[2].x, xh[2].y); o.z = *reinterpret_cast<uint32_t *>(&h);
+                    h = __floats2bfloat162_rn(xh[3].x, xh[3].y); o.w = *reinterpret_cast<uint32_t *>(&h);
                     *reinterpret_cast<uint4 *>(qdq + r * K + c) = o;
                 }
-                if (codes && !p.dst_rows) {
+            }
+            if (!codes) continue;
+            // the 4 scale codes of blocks kb0..kb0+3 on lanes 8j
+            uint32_t sw = sf_code | (__shfl_down_sync(0xffffffffu, sf_code, 2) << 8);
+            sw |= __shfl_down_sync(0xffffffffu, sw, 4) << 16;
+            if (!fanout) {
+                if (active) {
                     *reinterpret_cast<uint32_t *>(codes + r * (K >> 1) + (c >> 1)) = cw;
                     if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(scales + sf_offset(r, kb0, K)) = sw;
                 }
+                continue;
             }
-            if (codes && p.dst_rows) {
-                // fan-out: lane j < fanout fetches destination j of this row and
-                // stages its code / scale-atom row offsets in shared memory; the
-                // warp then writes the row's codes (128 contiguous bytes) and
-                // scale words to each destination.
-                if (lane < p.fanout) {
-                    const int64_t dst = p.dst_rows[r * p.fanout + lane];
-                    fan[warp][lane] = (dst >= 0 && dst < p.M_out) ? make_longlong2(dst * (K >> 1), sf_offset(dst, 0, K))
-                                               : make_longlong2(-1, 0);
+            // fan-out: stage the row's codes, one bulk copy per destination
+            uint32_t *slot = fstage[warp][fan_slot];
+            if (lane < fanout) ptx::bulk_wait_read<QFAN_SLOTS - 1>();
+            __syncwarp();
+            slot[lane] = cw;
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane < fanout) {
+                const int64_t dst = fdst[warp][i][lane];
+                if (dst >= 0 && dst < p.M_out) {
+                    ptx::bulk_store(codes + dst * (K >> 1) + (c0 >> 1), ptx::smem_u32(slot), code_bytes);
                 }
-                __syncwarp();
-                const int64_t sf_col_off = (kb0 >> 2) * 512;
-                for (int j = 0; j < p.fanout; ++j) {
-                    const longlong2 o = fan[warp][j];
-                    if (o.x < 0 || !active) continue;
-                    *reinterpret_cast<uint32_t *>(codes + o.x + (c >> 1)) = cw;
-                    if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(scales + o.y + sf_col_off) = sw;
-                }
-                __syncwarp();
+                ptx::bulk_commit();
+            }
+            fan_slot = (fan_slot + 1) % QFAN_SLOTS;
+            // scale words: lane l writes word l % 4 of destination l / 4 (+ 8 per round)
+            const uint32_t word = __shfl_sync(0xffffffffu, sw, (lane & 3) * 8);
+            const int64_t col = (c0 >> 4) + 4 * (lane & 3);       // first scale column of the word
+            for (int d = lane >> 2; d < fanout; d += 8) {
+                const int64_t dst = fdst[warp][i][d];
+                if (dst >= 0 && dst < p.M_out && col < (K >> 4))
+                    *reinterpret_cast<uint32_t *>(scales + sf_offset(dst, col, K)) = word;
             }
         }
         if (SCORE) {
             // at most QROWS / 8 = 4 rows were summed in binary32
 #pragma unroll
-            for (int k = 0; k < 8; ++k) { acc64[k] += (double)acc32[k]; acc32[k] = 0.0f; }
+            for (int k = 0; k < 4; ++k) {
+                acc64[2 * k] += (double)acc32[k].x;
+                acc64[2 * k + 1] += (double)acc32[k].y;
+                acc32[k] = make_float2(0.0f, 0.0f);
+            }
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty_bar[st]));
@@ -288,6 +325,7 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
             ++issued;
         }
     }
+    if (fanout && lane < fanout) ptx::bulk_wait_all();            // staged rows read and written
     if (threadIdx.x == 0) {
         // after an early exit, let every issued copy land before the CTA ends
         for (int j = it; j < issued; ++j)
@@ -299,7 +337,8 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
         __syncthreads();                                          // the stage ring is free: reuse it
         double *red = reinterpret_cast<double *>(qsm);            // [8 warps][256 channels]
 #pragma unroll
-        for (int i = 0; i < 8; ++i) red[warp * QCHUNK + lane * 8 + i] = acc64[i] + (double)acc32[i];
+        for (int i = 0; i < 8; ++i)
+            red[warp * QCHUNK + lane * 8 + i] = acc64[i] + (double)((i & 1) ? acc32[i >> 1].y : acc32[i >> 1].x);
         __syncthreads();
         int64_t ch = c0 + threadIdx.x;
         if (ch < K) {
@@ -458,7 +497,7 @@ __global__ void __launch_bounds__(256) k_rac_residual(
     if (m_valid) Me = min(Me, (int64_t)max(*m_valid, 0));
     if (r >= Me) return;
     const float s_t = *s_t_ptr;
-    const float r6 = block_r6(s_t);
+    const float2 r6 = recip_bracket(__fmul_rn(6.0f, s_t));
     const int nd = dst_rows ? fanout : 1;
     for (int j = lane; j < ld; j += 32) {
         __nv_bfloat16 outv = __float2bfloat16_rn(0.0f);
@@ -471,11 +510,11 @@ __global__ void __launch_bounds__(256) k_rac_residual(
             float m = 0.0f;
 #pragma unroll
             for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[i])), fabsf(bf16hi(w[i]))));
-            BlockScale bs = block_scale(m, s_t, r6);
+            const BlockConst b = block_const(block_scale_code(m, s_t, r6), s_t);
             int idx = (int)(ch & 15);
             uint32_t word = w[idx >> 1];
             float xv = (idx & 1) ? bf16hi(word) : bf16lo(word);
-            float R = __fsub_rn(xv, quant1_xhat(xv, bs));
+            float R = __fsub_rn(xv, element_xhat1(xv, b, s_t));
             outv = __float2bfloat16_rn(__fdiv_rn(R, s_t));
         }
         for (int d = 0; d < nd; ++d) {
@@ -631,20 +670,27 @@ static int64_t row_groups(int64_t M, int64_t rpc) { return std::max<int64_t>(1, 
 // Builds the TMA map over x ([rows_total x K] bf16, row stride ldx) and
 // launches k_quantize.  `fallback` is any valid 16-byte aligned device
 // address, used as the map's base when x has no rows (no copy is issued then).
+template <bool SCORE, bool QDQ>
+static nvfp4_status launch_quantize_t(const CUtensorMap &tm, const QuantParams &p, dim3 grid, size_t smem,
+                                      cudaStream_t st)
+{
+    static std::once_flag once[64];
+    static cudaError_t attr_err[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return check_launch("k_quantize: device");
+    std::call_once(once[dev], [&] {
+        attr_err[dev] = cudaFuncSetAttribute(k_quantize<SCORE, QDQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)QSMEM);
+    });
+    if (attr_err[dev] != cudaSuccess) return set_error(NVFP4_ERR_CUDA, "k_quantize: smem attribute: %s",
+                                                       cudaGetErrorString(attr_err[dev]));
+    k_quantize<SCORE, QDQ><<<grid, QTHREADS, smem, st>>>(tm, p);
+    return check_launch("k_quantize");
+}
+
 static nvfp4_status launch_quantize(bool score, const void *x, int64_t rows_total, const void *fallback,
                                     QuantParams &p, dim3 grid, cudaStream_t st)
 {
-    static bool attr_done[2][64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[score][dev]) {
-        cudaError_t e = score ? cudaFuncSetAttribute(k_quantize<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     (int)QSMEM)
-                              : cudaFuncSetAttribute(k_quantize<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     (int)QSMEM);
-        if (e != cudaSuccess) return check_launch("k_quantize: smem attribute");
-        attr_done[score][dev] = true;
-    }
     p.box_inner = (int)std::min<int64_t>(QCHUNK, p.K);
     CUtensorMap tm;
     const bool empty = rows_total <= 0 || x == nullptr;
@@ -653,9 +699,9 @@ static nvfp4_status launch_quantize(bool score, const void *x, int64_t rows_tota
                       CU_TENSOR_MAP_SWIZZLE_NONE))
         return set_error(NVFP4_ERR_CUDA, "k_quantize: tensor map encoding failed");
     const size_t smem = (size_t)QSTAGES * QROWS * p.box_inner * 2;
-    if (score) k_quantize<true><<<grid, QTHREADS, smem, st>>>(tm, p);
-    else k_quantize<false><<<grid, QTHREADS, smem, st>>>(tm, p);
-    return check_launch("k_quantize");
+    if (p.qdq) return launch_quantize_t<false, true>(tm, p, grid, smem, st);
+    if (score) return launch_quantize_t<true, false>(tm, p, grid, smem, st);
+    return launch_quantize_t<false, false>(tm, p, grid, smem, st);
 }
 
 }  // namespace nvfp4
@@ -754,15 +800,15 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
     }
     if (rac_k > 0) {
         size_t smem = (size_t)K * sizeof(unsigned long long);
-        static bool attr_set[64];
+        static std::once_flag once[64];
+        static cudaError_t attr_err[64];
         int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-            if (cudaFuncSetAttribute(k_select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, 16384 * 8) !=
-                cudaSuccess)
-                return check_launch("nvfp4_quantize: smem attribute");
-            attr_set[dev] = true;
-        }
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return check_launch("nvfp4_quantize: device");
+        std::call_once(once[dev], [&] {
+            attr_err[dev] = cudaFuncSetAttribute(k_select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, 16384 * 8);
+        });
+        if (attr_err[dev] != cudaSuccess)
+            return set_error(NVFP4_ERR_CUDA, "nvfp4_quantize: smem attribute: %s", cudaGetErrorString(attr_err[dev]));
         k_select_topk<<<1, 1024, smem, st>>>(score, (int)K, rac_k, sel_dev);
         if (check_launch("k_select_topk") != NVFP4_OK) return NVFP4_ERR_CUDA;
         if (M > 0) {
@@ -880,15 +926,18 @@ extern "C" nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_
                   "nvfp4_gather_weight_channels_cm: pointers must be 16-byte aligned");
     size_t smem = (size_t)ld * GCM_N * sizeof(float);
     {
-        static bool attr_done[64];
+        static std::once_flag once[64];
+        static cudaError_t attr_err[64];
         int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-            if (cudaFuncSetAttribute(k_gather_w_channels_cm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)(256 * GCM_N * sizeof(float))) != cudaSuccess)
-                return check_launch("nvfp4_gather_weight_channels_cm: smem attribute");
-            attr_done[dev] = true;
-        }
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            return check_launch("nvfp4_gather_weight_channels_cm: device");
+        std::call_once(once[dev], [&] {
+            attr_err[dev] = cudaFuncSetAttribute(k_gather_w_channels_cm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)(256 * GCM_N * sizeof(float)));
+        });
+        if (attr_err[dev] != cudaSuccess)
+            return set_error(NVFP4_ERR_CUDA, "nvfp4_gather_weight_channels_cm: smem attribute: %s",
+                             cudaGetErrorString(attr_err[dev]));
     }
     dim3 grid((unsigned)((N + GCM_N - 1) / GCM_N), (unsigned)E);
     k_gather_w_channels_cm<<<grid, 256, smem, (cudaStream_t)stream>>>(codes_cm_dev, scales_cm_dev, N, K, sel_dev, k,

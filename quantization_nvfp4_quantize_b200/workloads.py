@@ -58,6 +58,11 @@ CONFIGS = {
     # large MoE layer: T=16384, H=4096, I=1536, E=128, top-8 with skew, k = 128
     "moe_t16384_e128": LayerConfig("moe_t16384_e128", 16384, 4096, 1536, 128, 8, 128,
                                    round(0.01 * 4096), "lognormal", True),
+    # the large layer's shapes per expert (H=4096, I=1536, ~1024 routed rows
+    # per expert, k = 128) with 32 experts: small enough for detailed profiler
+    # captures (NVFP4 weights 340 MB, a few GB on the device)
+    "moe_t4096_h4096_e32": LayerConfig("moe_t4096_h4096_e32", 4096, 4096, 1536, 32, 8, 128,
+                                       round(0.01 * 4096), "lognormal", True),
 }
 
 CONFIG_ORDER = ["dense_64x256", "moe_t512_e8", "moe_t4096_e128", "qat_w4a16_e128",

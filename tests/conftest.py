@@ -34,3 +34,18 @@ def cuda():
     from quantization_nvfp4_quantize_b200 import _lib
     _lib.load()     # raises (fails the test) if the extension is not built
     return torch.device("cuda:0")
+
+
+def division_cases():
+    """Blocks of tests/golden/division_cases.txt as dicts: kind, s_t (binary32
+    bits), x (16 bf16 bit patterns), sf (E4M3 code), codes (16 E2M1 codes),
+    xhat (16 binary32 bit patterns)."""
+    rows = []
+    with open(os.path.join(GOLDEN, "division_cases.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            p = line.split()
+            rows.append(dict(kind=p[0], s_t=int(p[1], 16), x=[int(v, 16) for v in p[2:18]], sf=int(p[18], 16),
+                             codes=[int(c, 16) for c in p[19]], xhat=[int(v, 16) for v in p[20:36]]))
+    return rows

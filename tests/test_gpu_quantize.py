@@ -291,3 +291,80 @@ def test_fanout_skips_rows_beyond_m_out(cuda):
             d = dst[r, j]
             if d < m_out:
                 assert np.array_equal(codes[d], ref.codes[r])
+
+
+def _codes16(packed):
+    return [int(packed[i // 2] >> (4 * (i % 2)) & 15) for i in range(16)]
+
+
+def test_division_boundary_blocks_match_oracle(cuda):
+    """The stored blocks on which a reciprocal-multiply or double-rounded
+    shortcut would give other scale codes, element codes or dequantized
+    values (tests/golden/division_cases.txt): the kernels' codes, scales,
+    residual operand and fake-quantized values equal the stored ones."""
+    from conftest import division_cases
+    for c in division_cases():
+        x = np.zeros((1, 64), np.uint16)
+        x[0, :16] = c["x"]
+        s_t = np.array([c["s_t"]], np.uint32).view(np.float32)
+        st = torch.from_numpy(s_t.copy()).to(cuda)
+        q = api.quantize(to_bf16_dev(x, cuda), rac_k=16, s_t=st, want_score=True)
+        torch.cuda.synchronize()
+        assert unswizzle(q.scales, 1, 64)[0, 0] == c["sf"]
+        assert _codes16(q.codes.cpu().numpy()[0]) == c["codes"]
+        ref = oracle.quantize(x, s_t=float(s_t[0]))
+        sel = q.sel.cpu().numpy()[:16]
+        assert np.array_equal(np_u16(q.r_sel)[:, :16], oracle.rac_residual(ref.resid, ref.s_t, sel))
+        xh = np.array(c["xhat"], np.uint32).view(np.float32)
+        assert np.array_equal(ref.xhat[0, :16].view(np.uint32), c["xhat"])
+        del xh
+
+
+def _near_boundary_groups(rng, G, rows, cols):
+    """G weight tensors whose blocks sit next to the encoders' rounding
+    boundaries: each block has a maximum whose scale quotient a/(6 s_t) lies
+    near an E4M3 midpoint or value, and elements at the bf16 values nearest
+    to an E2M1 threshold times the block scale.  The tensor scale comes from
+    one planted maximum per tensor."""
+    e4 = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    thr = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    out = np.empty((G, rows, cols), np.uint16)
+    nb = rows * cols // 16
+    for g in range(G):
+        A = float(oracle.bf16_to_f32(oracle.f32_to_bf16(np.array([rng.uniform(1.0, 2.0) * 2.0 ** rng.integers(-8, 8)],
+                                                                np.float32)))[0])
+        s_t = np.float32(np.float32(A) / np.float32(2688.0))
+        c = rng.integers(0x08, 0x7E, nb)
+        mid = np.where(rng.random(nb) < 0.5, (e4[c] + e4[c + 1]) / 2, e4[c])
+        amax_b = np.minimum(6.0 * mid * float(s_t), A)
+        d = (e4[c].astype(np.float32) * s_t).astype(np.float64)
+        t = thr[rng.integers(0, 7, (nb, 15))] * np.where(rng.random((nb, 15)) < 0.5, -1.0, 1.0)
+        vals = np.concatenate([amax_b[:, None], t * d[:, None]], axis=1)
+        blk = oracle.f32_to_bf16(vals.astype(np.float32)).reshape(rows, cols)
+        blk[0, 0] = oracle.f32_to_bf16(np.array([A], np.float32))[0]
+        out[g] = blk
+    return out
+
+
+def test_near_boundary_sweep_matches_oracle(cuda):
+    """About a million blocks built at the encoders' rounding boundaries, as
+    per-tensor weight fake quantization (each tensor its own s_t): codes,
+    scale bytes and bf16 dequantized values bit-exact against the oracle, and
+    the activation path (given s_t, with scores) gives the same codes."""
+    rng = np.random.default_rng(123)
+    G, rows, cols = 1024, 64, 256
+    w = _near_boundary_groups(rng, G, rows, cols)
+    wq, s_t, codes, scales = api.qdq_weights(to_bf16_dev(w, cuda), want_qdq=True, want_packed=True)
+    torch.cuda.synchronize()
+    wq, s_t, codes, scales = np_u16(wq), s_t.cpu().numpy(), codes.cpu().numpy(), scales.cpu().numpy()
+    for g in range(G):
+        ref_bf16, ref_s, ref = oracle.qdq(w[g])
+        assert s_t[g] == np.float32(ref_s)
+        assert np.array_equal(codes[g], ref.codes), g
+        assert np.array_equal(oracle.unswizzle_scales(scales[g], rows, cols), ref.sf), g
+        assert np.array_equal(wq[g], ref_bf16), g
+    for g in range(0, G, 97):
+        q = api.quantize(to_bf16_dev(w[g], cuda), rac_k=32, s_t=torch.tensor([s_t[g]], device=cuda),
+                         want_score=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(q.codes.cpu().numpy(), codes[g])

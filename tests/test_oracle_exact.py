@@ -4,31 +4,17 @@ OCP E2M1 / E4M3 code tables), on random blocks and on stored blocks
 (tests/golden/division_cases.txt) chosen so that a reciprocal-multiply
 scale or element step, or a double-rounded dequantization, would give
 other codes or values."""
-import os
-
 import numpy as np
 import pytest
 
 import oracle
-from conftest import GOLDEN
+from conftest import division_cases
 from exact_fp import quantize_block_exact, f32_bits_to_fraction
 
 F = np.float32
 
 
-def _cases():
-    rows = []
-    with open(os.path.join(GOLDEN, "division_cases.txt")) as f:
-        for line in f:
-            if line.startswith("#") or not line.strip():
-                continue
-            p = line.split()
-            rows.append(dict(kind=p[0], s_t=int(p[1], 16), x=[int(v, 16) for v in p[2:18]], sf=int(p[18], 16),
-                             codes=[int(c, 16) for c in p[19]], xhat=[int(v, 16) for v in p[20:36]]))
-    return rows
-
-
-CASES = _cases()
+CASES = division_cases()
 
 
 def _oracle_block(x_bits, s_t_bits):
