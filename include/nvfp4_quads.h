@@ -372,6 +372,24 @@ NVFP4_API nvfp4_status moe_gather_rows_bf16(const void *x_dev, int64_t T, int64_
                                             int64_t ld_out, int64_t M_out, void *stream);
 
 /* --------------------------------------------------------------------------
+ * nvfp4_debug_gemm_wait_expiry -- test hook for the bounded device waits of
+ * the grouped GEMM (the pages have no counterpart).  Runs
+ * moe_w4a4_grouped_gemm_rac in its 1-SM shape (seg_align 128, no RAC) with
+ * every mbarrier wait bounded by wait_limit_ns (1 ms .. 1 s), and with the
+ * MMA issuer withholding the "accumulator ready" signal of the first tile
+ * (it drains its MMAs itself), so the epilogue's wait runs out.  Expected
+ * outcome: *dev_status = NVFP4_ERR_TIMEOUT, every copy and MMA drained, tensor
+ * memory freed, the kernel returns and the context stays usable; the output
+ * of the withheld tile is not written.  Arguments as for
+ * moe_w4a4_grouped_gemm_rac; dev_status is required.
+ * -------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_debug_gemm_wait_expiry(
+    const uint8_t *a_codes_dev, const uint8_t *a_scales_dev, const float *a_s_t_dev, int64_t M_pad_max,
+    const uint8_t *b_codes_dev, const uint8_t *b_scales_dev, const float *b_s_t_dev, int64_t N, int64_t K, int32_t E,
+    const int32_t *offsets_dev, int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev,
+    void *out_dev, int64_t ld_out, int32_t *dev_status, int64_t wait_limit_ns, void *stream);
+
+/* --------------------------------------------------------------------------
  * nvfp4_debug_encode -- runs the library's element and scale encoders on n
  * arbitrary floats (for validation against an independent definition):
  *   e2m1_dev[i] = E2M1 code of in[i] (nearest even, saturating, sign bit

@@ -51,6 +51,9 @@ SIGNATURES = {
     "moe_gather_rows_bf16": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int32, c_void_p, c_int64,
                                        c_int64, c_void_p]),
     "nvfp4_debug_encode": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
+    "nvfp4_debug_gemm_wait_expiry": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
+                                               c_int64, c_int64, c_int32, c_void_p, c_int32, c_void_p, c_void_p,
+                                               c_void_p, c_int64, c_void_p, c_int64, c_void_p]),
 }
 
 STATUS_NAMES = {0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_ALIGNMENT",

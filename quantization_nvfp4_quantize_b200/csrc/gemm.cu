@@ -85,8 +85,9 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0, SF_COL = 256, SF_STRIDE = 48;  // scale buffer of stage s: SF_COL + 48 s
 constexpr int PROD_A_WARP = 0, MMA_WARP = 1, PROD_B_WARP = 2, COPY_WARP = 3, EPI_WARP0 = 4;
 constexpr int MAX_E = 256;
-constexpr uint64_t TIMEOUT_NS = 1000000000ull;
+constexpr uint64_t TIMEOUT_NS = 1000000000ull;    // default bound of every mbarrier wait (1 s)
 constexpr uint32_t STAGING_BYTES = EPI_WARPS * 32 * 32 * 4;   // one 32 x 32 f32 transpose tile per epilogue warp
+constexpr int BOX_ROWS = 128;                   // rows per operand TMA box (128-byte rows)
 
 template <bool PAIR>
 struct Geo {
@@ -123,6 +124,9 @@ struct Params {
     void *out;
     int64_t ld_out;
     unsigned int *amax_out;    // SwiGLU: max |h| (float bits), or null
+    int l2_hints;              // scatter-add: stream A with evict-first loads, reduce into the output with evict-last
+    uint64_t wait_limit_ns;    // bound of every mbarrier wait
+    int debug_withhold_acc;    // test hook: no "accumulator ready" signal for the first tile (1-SM shape)
     int32_t *dev_status;
 };
 
@@ -141,7 +145,7 @@ struct Shared {
 
 // Bounded wait; returns false on abort or timeout (then sets the abort flag).
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                         int32_t *dev_status, bool ignore_abort = false)
+                                         int32_t *dev_status, uint64_t limit_ns, bool ignore_abort = false)
 {
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
@@ -150,7 +154,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
             if (!ignore_abort && *abort_flag) return false;
             uint64_t now = globaltimer_ns();
             if (t0 == 0) t0 = now;
-            else if (now - t0 > TIMEOUT_NS) {
+            else if (now - t0 > limit_ns) {
                 *abort_flag = 1;
                 report_status(dev_status, NVFP4_ERR_TIMEOUT);
                 return false;
@@ -260,6 +264,10 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             const uint32_t mult = PAIR ? 2u : 1u;
             const uint32_t tx_fp4 = mult * (role_a ? (A_BYTES + SFA_BYTES) : (G::B_LOCAL + SFB_BYTES));
             const uint32_t tx_rac = mult * (role_a ? A_BYTES : G::B_LOCAL);
+            // the scatter-add GEMM reads each A tile once per group of n-tiles:
+            // let those lines leave L2 first so the output band stays resident
+            const bool hint_a = p.l2_hints != 0;
+            const uint64_t pol_a = ptx::policy_evict_first();
             uint32_t stage = 0, phase = 0;
             uint32_t issued_phase[STAGES];
             bool issued[STAGES];
@@ -280,7 +288,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                 const int64_t sfb_off0 = sfb_e + (int64_t)(nrow0 / 128) * (p.K / 64) * 512;
                 const int64_t sfb_off1 = sfb_e + (int64_t)(nrow1 / 128) * (p.K / 64) * 512;
                 for (int kb = 0; kb < nkb + nrk; ++kb) {
-                    if (!wait_bar(ptx::smem_u32(&sh->empty[stage]), phase ^ 1u, abort_flag, p.dev_status)) {
+                    if (!wait_bar(ptx::smem_u32(&sh->empty[stage]), phase ^ 1u, abort_flag, p.dev_status, p.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
@@ -295,7 +303,15 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                     if (PAIR) {
                         const uint32_t lfb = ptx::mapa_shared(fb, 0);     // the leader's barrier
                         const int browr = rank ? brow1 : brow0;
-                        if (role_a) {
+                        if (role_a && hint_a) {
+                            if (fp4) {
+                                ptx::tma_load_2d_pair_hint(ptx::smem_u32(sa), &tm_a, kb * 128, arow, lfb, pol_a);
+                                ptx::tma_load_2d_pair_hint(ptx::smem_u32(ssfa), &tm_sfa, 0, sf_row(sfa_off + kb * 2048),
+                                                           lfb, pol_a);
+                            } else {
+                                ptx::tma_load_2d_pair_hint(ptx::smem_u32(sa), &tm_ra, rk * 64, arow, lfb, pol_a);
+                            }
+                        } else if (role_a) {
                             if (fp4) {
                                 ptx::tma_load_2d_pair(ptx::smem_u32(sa), &tm_a, kb * 128, arow, lfb);
                                 ptx::tma_load_2d_pair(ptx::smem_u32(ssfa), &tm_sfa, 0, sf_row(sfa_off + kb * 2048), lfb);
@@ -312,8 +328,11 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                         }
                     } else if (role_a) {
                         if (fp4) {
-                            ptx::tma_load_2d(ptx::smem_u32(sa), &tm_a, kb * 128, m0, fb);
+                            if (hint_a) ptx::tma_load_2d_hint(ptx::smem_u32(sa), &tm_a, kb * 128, m0, fb, pol_a);
+                            else ptx::tma_load_2d(ptx::smem_u32(sa), &tm_a, kb * 128, m0, fb);
                             ptx::bulk_load(ptx::smem_u32(ssfa), p.a_scales + sfa_off + kb * 2048, SFA_BYTES, fb);
+                        } else if (hint_a) {
+                            ptx::tma_load_2d_hint(ptx::smem_u32(sa), &tm_ra, rk * 64, m0, fb, pol_a);
                         } else {
                             ptx::tma_load_2d(ptx::smem_u32(sa), &tm_ra, rk * 64, m0, fb);
                         }
@@ -337,7 +356,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                 if (!PAIR || leader) {
                     for (int s = 0; s < STAGES; ++s)
                         if (issued[s])
-                            wait_bar(ptx::smem_u32(&sh->full[s]), issued_phase[s], abort_flag, p.dev_status, true);
+                            wait_bar(ptx::smem_u32(&sh->full[s]), issued_phase[s], abort_flag, p.dev_status, p.wait_limit_ns, true);
                 } else {
                     // the peer's copies complete on the leader's barriers: give them 100 us
                     const uint64_t t0 = globaltimer_ns();
@@ -356,15 +375,15 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             bool issued_any = false;
             int iter = 0;
             for (int t = unit; ok && t < total; t += n_units, ++iter) {
-                if (!wait_bar(ptx::smem_u32(&sh->tmem_empty), (uint32_t)(iter & 1) ^ 1u, abort_flag, p.dev_status)) {
+                if (!wait_bar(ptx::smem_u32(&sh->tmem_empty), (uint32_t)(iter & 1) ^ 1u, abort_flag, p.dev_status, p.wait_limit_ns)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
                 for (int kb = 0; kb < nkb && ok; ++kb) {
                     // the stage's data has landed and its scale factors are in TMEM
-                    if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status) ||
-                        !wait_bar(ptx::smem_u32(&sh->sf_full[stage]), phase, abort_flag, p.dev_status)) {
+                    if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status, p.wait_limit_ns) ||
+                        !wait_bar(ptx::smem_u32(&sh->sf_full[stage]), phase, abort_flag, p.dev_status, p.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
@@ -393,14 +412,14 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                     // the FP4 MMAs to complete first
                     if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->drain), 1);
                     else ptx::tc_commit(ptx::smem_u32(&sh->drain));
-                    if (!wait_bar(ptx::smem_u32(&sh->drain), drain_phase, abort_flag, p.dev_status)) { ok = false; }
+                    if (!wait_bar(ptx::smem_u32(&sh->drain), drain_phase, abort_flag, p.dev_status, p.wait_limit_ns)) { ok = false; }
                     drain_phase ^= 1u;
                     ptx::tc_fence_after();
                 }
                 if (ok && nrk > 0) {
                     for (int rk = 0; rk < nrk && ok; ++rk) {
-                        if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status) ||
-                            !wait_bar(ptx::smem_u32(&sh->sf_full[stage]), phase, abort_flag, p.dev_status)) {
+                        if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status, p.wait_limit_ns) ||
+                            !wait_bar(ptx::smem_u32(&sh->sf_full[stage]), phase, abort_flag, p.dev_status, p.wait_limit_ns)) {
                             ok = false;
                             break;
                         }
@@ -421,7 +440,15 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     }
                 }
-                if (ok) {
+                if (ok && !PAIR && p.debug_withhold_acc && iter == 0) {
+                    // test hook: withhold the tile's "accumulator ready" signal so
+                    // the epilogue's bounded wait runs out; the MMAs are drained
+                    // here instead, before any thread can release TMEM
+                    ptx::tc_commit(ptx::smem_u32(&sh->drain));
+                    if (!wait_bar(ptx::smem_u32(&sh->drain), drain_phase, abort_flag, p.dev_status, p.wait_limit_ns))
+                        ok = false;
+                    drain_phase ^= 1u;
+                } else if (ok) {
                     if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->tmem_full), 3);
                     else ptx::tc_commit(ptx::smem_u32(&sh->tmem_full));
                 }
@@ -430,7 +457,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                 // let every issued MMA finish before TMEM is released
                 if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->drain), 1);
                 else ptx::tc_commit(ptx::smem_u32(&sh->drain));
-                wait_bar(ptx::smem_u32(&sh->drain), drain_phase, abort_flag, p.dev_status, true);
+                wait_bar(ptx::smem_u32(&sh->drain), drain_phase, abort_flag, p.dev_status, p.wait_limit_ns, true);
             }
         }
         __syncwarp();
@@ -444,7 +471,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             bool ok = true, issued_any = false;
             for (int t = unit; ok && t < total; t += n_units) {
                 for (int kb = 0; kb < nkb + nrk; ++kb) {
-                    if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status)) {
+                    if (!wait_bar(ptx::smem_u32(&sh->full[stage]), phase, abort_flag, p.dev_status, p.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
@@ -479,7 +506,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                 // copies still in flight complete before TMEM is released
                 if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->cp_drain), 1);
                 else ptx::tc_commit(ptx::smem_u32(&sh->cp_drain));
-                wait_bar(ptx::smem_u32(&sh->cp_drain), 0, abort_flag, p.dev_status, true);
+                wait_bar(ptx::smem_u32(&sh->cp_drain), 0, abort_flag, p.dev_status, p.wait_limit_ns, true);
             }
         }
         __syncwarp();
@@ -497,7 +524,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
         int iter = 0;
         for (int t = unit; t < total; t += n_units, ++iter) {
             bool ok = true;
-            if (lane == 0) ok = wait_bar(ptx::smem_u32(&sh->tmem_full), (uint32_t)(iter & 1), abort_flag, p.dev_status);
+            if (lane == 0) ok = wait_bar(ptx::smem_u32(&sh->tmem_full), (uint32_t)(iter & 1), abort_flag, p.dev_status, p.wait_limit_ns);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
             ptx::tc_fence_after();
@@ -563,6 +590,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                 // vector stores (store) or vector add-reductions (scatter-add
                 // into the token rows).  Padding rows are never written.
                 const bool scatter = p.epilogue == MOE_EPI_SCATTER_ADD_F32;
+                const bool hint_y = p.l2_hints != 0;
+                const uint64_t pol_y = ptx::policy_evict_last();
                 const bool has_row = token >= 0;
                 const float mul = scatter ? (has_row ? __fmul_rn(scale, p.row_gate[r]) : 0.0f) : scale;
                 const int32_t orow = scatter ? token : (int32_t)r;
@@ -587,7 +616,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                         const float4 val = tile[rr * 8 + (jj ^ (rr & 7))];
                         if (valid_r) {
                             float *dst = out_base + (int64_t)orow_r * p.ld_out + ch * 32 + jj * 4;
-                            if (scatter) ptx::red_add_v4_f32(dst, val);
+                            if (scatter && hint_y) ptx::red_add_v4_f32_hint(dst, val, pol_y);
+                            else if (scatter) ptx::red_add_v4_f32(dst, val);
                             else ptx::st_v4_f32(dst, val);
                         }
                     }
@@ -666,6 +696,8 @@ static nvfp4_status dispatch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, c
         if (g > 0 && n_tiles % g == 0) n_group = g;
     }
     p.n_group = n_group;
+    p.l2_hints = epilogue == MOE_EPI_SCATTER_ADD_F32 ? 1 : 0;
+    if (const char *env = getenv("NVFP4_GEMM_L2HINTS")) p.l2_hints = p.l2_hints && atoi(env) != 0;
     const int64_t max_tiles = (M_pad_max / seg_align) * n_tiles;
     const bool swiglu = epilogue == MOE_EPI_SWIGLU_BF16;
     if (pair) {
@@ -685,12 +717,12 @@ static nvfp4_status dispatch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, c
 
 using namespace nvfp4;
 
-extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
+static nvfp4_status gemm_rac(
     const uint8_t *a_codes_dev, const uint8_t *a_scales_dev, const float *a_s_t_dev, int64_t M_pad_max,
     const uint8_t *b_codes_dev, const uint8_t *b_scales_dev, const float *b_s_t_dev, int64_t N, int64_t K, int32_t E,
     const int32_t *offsets_dev, int32_t seg_align, int32_t rac_ld, const void *rho_dev, const void *w_sel_dev,
     int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev, void *out_dev, int64_t ld_out,
-    float *amax_out_dev, int32_t *dev_status, void *stream)
+    float *amax_out_dev, int32_t *dev_status, void *stream, uint64_t wait_limit_ns, int debug_withhold_acc)
 {
     using namespace nvfp4::gemm;
     cudaStream_t st = (cudaStream_t)stream;
@@ -731,14 +763,14 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
     CUtensorMap tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     bool ok = make_tmap_2d(&tm_a, a_codes_dev, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)M_pad_max,
-                           (uint64_t)K / 2, 128, 128, sw) &&
+                           (uint64_t)K / 2, 128, BOX_ROWS, sw) &&
               make_tmap_2d(&tm_b, b_codes_dev, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)E * N,
-                           (uint64_t)K / 2, 128, 128, sw);
+                           (uint64_t)K / 2, 128, BOX_ROWS, sw);
     if (ok && rac_ld > 0) {
         ok = make_tmap_2d(&tm_ra, rho_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)rac_ld, (uint64_t)M_pad_max,
-                          (uint64_t)rac_ld * 2, 64, 128, sw) &&
+                          (uint64_t)rac_ld * 2, 64, BOX_ROWS, sw) &&
              make_tmap_2d(&tm_rb, w_sel_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)rac_ld, (uint64_t)E * N,
-                          (uint64_t)rac_ld * 2, 64, 128, sw);
+                          (uint64_t)rac_ld * 2, 64, BOX_ROWS, sw);
     } else {
         tm_ra = tm_a;
         tm_rb = tm_b;
@@ -775,10 +807,37 @@ extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
     p.out = out_dev;
     p.ld_out = ld_out;
     p.amax_out = (epilogue == MOE_EPI_SWIGLU_BF16) ? reinterpret_cast<unsigned int *>(amax_out_dev) : nullptr;
+    p.wait_limit_ns = wait_limit_ns;
+    p.debug_withhold_acc = debug_withhold_acc;
     p.dev_status = dev_status;
     if (p.amax_out && cudaMemsetAsync(p.amax_out, 0, sizeof(float), st) != cudaSuccess)
         return check_launch("moe_w4a4_grouped_gemm_rac: memset");
     return dispatch(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, M_pad_max, seg_align, st);
+}
+
+extern "C" nvfp4_status moe_w4a4_grouped_gemm_rac(
+    const uint8_t *a_codes_dev, const uint8_t *a_scales_dev, const float *a_s_t_dev, int64_t M_pad_max,
+    const uint8_t *b_codes_dev, const uint8_t *b_scales_dev, const float *b_s_t_dev, int64_t N, int64_t K, int32_t E,
+    const int32_t *offsets_dev, int32_t seg_align, int32_t rac_ld, const void *rho_dev, const void *w_sel_dev,
+    int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev, void *out_dev, int64_t ld_out,
+    float *amax_out_dev, int32_t *dev_status, void *stream)
+{
+    return gemm_rac(a_codes_dev, a_scales_dev, a_s_t_dev, M_pad_max, b_codes_dev, b_scales_dev, b_s_t_dev, N, K, E,
+                    offsets_dev, seg_align, rac_ld, rho_dev, w_sel_dev, epilogue, row_token_dev, row_gate_dev, out_dev,
+                    ld_out, amax_out_dev, dev_status, stream, nvfp4::gemm::TIMEOUT_NS, 0);
+}
+
+extern "C" nvfp4_status nvfp4_debug_gemm_wait_expiry(
+    const uint8_t *a_codes_dev, const uint8_t *a_scales_dev, const float *a_s_t_dev, int64_t M_pad_max,
+    const uint8_t *b_codes_dev, const uint8_t *b_scales_dev, const float *b_s_t_dev, int64_t N, int64_t K, int32_t E,
+    const int32_t *offsets_dev, int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev,
+    void *out_dev, int64_t ld_out, int32_t *dev_status, int64_t wait_limit_ns, void *stream)
+{
+    NVFP4_REQUIRE(dev_status && wait_limit_ns >= 1000000 && wait_limit_ns <= 1000000000ll, NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_debug_gemm_wait_expiry: needs dev_status and 1 ms <= wait_limit_ns <= 1 s");
+    return gemm_rac(a_codes_dev, a_scales_dev, a_s_t_dev, M_pad_max, b_codes_dev, b_scales_dev, b_s_t_dev, N, K, E,
+                    offsets_dev, 128, 0, nullptr, nullptr, epilogue, row_token_dev, row_gate_dev, out_dev, ld_out,
+                    nullptr, dev_status, stream, (uint64_t)wait_limit_ns, 1);
 }
 
 extern "C" nvfp4_status moe_bf16_grouped_gemm(
@@ -822,9 +881,9 @@ extern "C" nvfp4_status moe_bf16_grouped_gemm(
     CUtensorMap tm_ra, tm_rb;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     const bool ok = make_tmap_2d(&tm_ra, a_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)K, (uint64_t)M_pad_max,
-                                 (uint64_t)lda * 2, 64, 128, sw) &&
+                                 (uint64_t)lda * 2, 64, BOX_ROWS, sw) &&
                     make_tmap_2d(&tm_rb, b_dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)K, (uint64_t)E * N,
-                                 (uint64_t)K * 2, 64, 128, sw);
+                                 (uint64_t)K * 2, 64, BOX_ROWS, sw);
     NVFP4_REQUIRE(ok, NVFP4_ERR_CUDA, "moe_bf16_grouped_gemm: tensor map encoding failed");
 
     Params p{};
@@ -840,6 +899,7 @@ extern "C" nvfp4_status moe_bf16_grouped_gemm(
     p.out = out_dev;
     p.ld_out = ld_out;
     p.amax_out = (epilogue == MOE_EPI_SWIGLU_BF16) ? reinterpret_cast<unsigned int *>(amax_out_dev) : nullptr;
+    p.wait_limit_ns = TIMEOUT_NS;
     p.dev_status = dev_status;
     if (p.amax_out && cudaMemsetAsync(p.amax_out, 0, sizeof(float), st) != cudaSuccess)
         return check_launch("moe_bf16_grouped_gemm: memset");

@@ -27,12 +27,16 @@
 
 namespace nvfp4 {
 
-constexpr int QTHREADS = 256;
-constexpr int QCHUNK = 256;           // channels per CTA column chunk
+constexpr int QWORKERS = 8;           // quantizing warps per CTA
+constexpr int QTHREADS = (QWORKERS + 1) * 32;   // + one TMA producer warp
+constexpr int QCHUNK = 256;           // channels per CTA column chunk (one 512-byte tile row)
 constexpr int QCTAS_PER_SM = 3;       // resident CTAs per SM the grid is sized for (one wave)
 constexpr int QSTAGES = 4;            // TMA tile ring depth
 constexpr int QROWS = 32;             // rows per TMA tile
-constexpr uint32_t QSMEM = QSTAGES * QROWS * QCHUNK * 2;   // 64 KB of tiles per CTA
+constexpr int QRPW = QROWS / QWORKERS;   // tile rows per worker warp
+constexpr uint32_t QPITCH = QCHUNK * 2;  // bytes per tile row
+constexpr uint32_t QTILE = QPITCH * QROWS;
+constexpr uint32_t QSMEM = QSTAGES * QTILE;   // 64 KB of tiles per CTA
 
 // -------------------------------------------------------------------- amax
 
@@ -133,36 +137,42 @@ __device__ __forceinline__ bool qwait(uint32_t bar, uint32_t parity, volatile in
 
 constexpr int QFAN_SLOTS = 4;         // per-warp ring of staged code rows for the fan-out bulk stores
 
-// One CTA = 8 warps on one 256-channel column chunk and one range of rows.
-// Thread 0 streams 32-row x 256-channel bf16 tiles (16 KB) through a 4-stage
-// shared-memory ring with TMA; warp w quantizes tile rows w, w+8, w+16, w+24,
-// each lane 8 channels (a lane pair is one 16-element block).  Arithmetic on
-// element pairs uses the packed f32x2 instructions.
+// Byte offset of scale entry (r, c) in the scale-factor layout, 32-bit
+// (callers keep rows x K/16 below 2^31).
+__device__ __forceinline__ uint32_t sf_off32(uint32_t r, uint32_t c, uint32_t K)
+{
+    return ((r >> 7) * (K >> 6) + (c >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (c & 3u);
+}
+
+// One CTA = 8 worker warps on one 256-channel column chunk and one range of
+// rows, plus a producer warp whose lane 0 streams 32-row x 256-channel bf16
+// tiles (16 KB, zero-filled past K) through a 4-stage shared-memory ring with
+// TMA.  Worker w quantizes tile rows w, w+8, w+16, w+24, each lane 8 channels
+// (a lane pair is one 16-element block).
 //   SCORE  accumulate the channels' residual sums of squares
 //   QDQ    write bf16(xhat) (weight fake quantization)
 // With dst_rows, the codes of a row (128 contiguous bytes per warp) are staged
 // in shared memory and written to each destination row by one bulk copy per
 // destination; the scale words go out as 4-byte stores, one per lane.
+// Offsets inside a tensor are 32-bit (the host checks the sizes).
 template <bool SCORE, bool QDQ>
 __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __grid_constant__ CUtensorMap tm_x,
                                                                      QuantParams p)
 {
-    extern __shared__ __align__(128) uint8_t qsm[];              // QSTAGES x QROWS x box_inner bf16
+    extern __shared__ __align__(128) uint8_t qsm[];              // QSTAGES x QROWS x 256 bf16
     __shared__ uint64_t full_bar[QSTAGES], empty_bar[QSTAGES];
     __shared__ int abort_sm;
     __shared__ float4 btab[128];                                  // per E4M3 code: d, rlo, rhi, sf_h2
-    __shared__ int32_t fdst[QTHREADS / 32][QROWS / (QTHREADS / 32)][32];      // fan-out rows of a warp's 4 rows
-    __shared__ __align__(128) uint32_t fstage[QTHREADS / 32][QFAN_SLOTS][32]; // staged code rows
+    __shared__ int32_t fdst[QWORKERS][QRPW][32];                  // fan-out rows of a warp's 4 rows
+    __shared__ __align__(128) uint32_t fstage[QWORKERS][QFAN_SLOTS][32];   // staged code rows
     volatile int *abort_flag = &abort_sm;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = blockIdx.z;
-    const int64_t K = p.K;
-    const int64_t c0 = (int64_t)blockIdx.x * QCHUNK;
-    const int64_t c = c0 + lane * 8;                              // first channel of this lane
+    const uint32_t K = (uint32_t)p.K;
+    const uint32_t c0 = blockIdx.x * QCHUNK;
+    const uint32_t c = c0 + lane * 8;                             // first channel of this lane
     const bool active = c < K;
-    const uint32_t pitch = (uint32_t)p.box_inner * 2u;            // bytes per tile row in shared memory
-    const uint32_t tile_bytes = pitch * QROWS;
 
     const float s_t = p.s_t_in ? p.s_t_in[g] : tensor_scale_from_amax(__uint_as_float(p.amax_bits[g]));
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.s_t_out) p.s_t_out[g] = s_t;
@@ -170,15 +180,17 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
 
     int64_t Me = p.M;
     if (p.m_valid) Me = min(Me, (int64_t)max(*p.m_valid, 0));
-    const int64_t r0 = (int64_t)blockIdx.y * p.rows_per_cta;
-    const int64_t r1 = min(Me, r0 + p.rows_per_cta);
-    const int n_iter = r1 > r0 ? (int)((r1 - r0 + QROWS - 1) / QROWS) : 0;
+    const int64_t r0l = (int64_t)blockIdx.y * p.rows_per_cta;
+    const int64_t r1l = min(Me, r0l + p.rows_per_cta);
+    const int n_iter = r1l > r0l ? (int)((r1l - r0l + QROWS - 1) / QROWS) : 0;
+    const uint32_t r0 = (uint32_t)r0l, r1 = (uint32_t)max(r1l, r0l);
     const int64_t row_base = (int64_t)g * p.M;                   // row of this group in the tensor map
 
     uint8_t *codes = p.codes ? p.codes + g * p.codes_gstride : nullptr;
     uint8_t *scales = p.scales ? p.scales + g * p.scales_gstride : nullptr;
     __nv_bfloat16 *qdq = QDQ ? p.qdq + g * p.qdq_gstride : nullptr;
     const int fanout = p.dst_rows ? p.fanout : 0;
+    const uint32_t M_out = (uint32_t)p.M_out;
 
     // E4M3 code -> the block's constants: a block scale takes at most 127
     // values per tensor, so each is computed once here rather than per block.
@@ -189,23 +201,13 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
     if (threadIdx.x == 0) {
         for (int st = 0; st < QSTAGES; ++st) {
             ptx::mbar_init(ptx::smem_u32(&full_bar[st]), 1);
-            ptx::mbar_init(ptx::smem_u32(&empty_bar[st]), QTHREADS / 32);
+            ptx::mbar_init(ptx::smem_u32(&empty_bar[st]), QWORKERS);
         }
         abort_sm = 0;
         ptx::fence_mbar_init();
         ptx::fence_proxy_async_smem();
     }
     __syncthreads();
-    int issued = 0;                                               // thread 0 only
-    if (threadIdx.x == 0) {
-        ptx::prefetch_tmap(&tm_x);
-        for (; issued < min(n_iter, QSTAGES); ++issued) {
-            const uint32_t fb = ptx::smem_u32(&full_bar[issued]);
-            ptx::mbar_arrive_expect_tx(fb, tile_bytes);
-            ptx::tma_load_2d(ptx::smem_u32(qsm + issued * tile_bytes), &tm_x, (int32_t)c0,
-                             (int32_t)(row_base + r0 + (int64_t)issued * QROWS), fb);
-        }
-    }
 
     float2 acc32[4];
     double acc64[8];
@@ -214,137 +216,147 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc64[i] = 0.0;
 
-    const int64_t kb0 = c >> 4;                 // first block of the lane octet's 4-block group (lanes 8j)
-    const uint32_t code_bytes = (uint32_t)(min((int64_t)QCHUNK, K - c0) / 2);   // one row's codes in this chunk
-    int fan_slot = 0;
-    int it = 0;
-    for (; it < n_iter; ++it) {
-        const int st = it % QSTAGES;
-        const uint32_t ph = (uint32_t)(it / QSTAGES) & 1u;
-        bool ok = true;
-        if (lane == 0) ok = qwait(ptx::smem_u32(&full_bar[st]), ph, abort_flag, p.dev_status);
-        if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
-        const uint8_t *tile = qsm + st * tile_bytes;
-        const int64_t rt = r0 + (int64_t)it * QROWS;             // first row of the tile
-        if (fanout) {
-            // this warp's 4 rows x fanout destinations, fetched once per tile
-            for (int e = lane; e < (QROWS / (QTHREADS / 32)) * fanout; e += 32) {
-                const int i = e / fanout, j = e - i * fanout;
-                const int64_t r = rt + warp + i * (QTHREADS / 32);
-                fdst[warp][i][j] = r < r1 ? p.dst_rows[r * fanout + j] : -1;
+    if (warp == QWORKERS) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            ptx::prefetch_tmap(&tm_x);
+            int issued = 0;
+            for (int it = 0; it < n_iter; ++it) {
+                const int st = it % QSTAGES;
+                // the stage's previous tile has been released by every worker
+                if (it >= QSTAGES &&
+                    !qwait(ptx::smem_u32(&empty_bar[st]), ((uint32_t)(it / QSTAGES) & 1u) ^ 1u, abort_flag,
+                           p.dev_status))
+                    break;
+                const uint32_t fb = ptx::smem_u32(&full_bar[st]);
+                ptx::mbar_arrive_expect_tx(fb, QTILE);
+                ptx::tma_load_2d(ptx::smem_u32(qsm + st * QTILE), &tm_x, (int32_t)c0,
+                                 (int32_t)(row_base + r0l + (int64_t)it * QROWS), fb);
+                ++issued;
+            }
+            // every issued copy lands before the CTA ends (each stage's last
+            // tile: its phase is the barrier's latest)
+            for (int j = max(0, issued - QSTAGES); j < issued; ++j)
+                qwait(ptx::smem_u32(&full_bar[j % QSTAGES]), (uint32_t)(j / QSTAGES) & 1u, abort_flag, p.dev_status,
+                      true);
+        }
+    } else {
+        // -------------------------------------------------------- workers
+        const uint32_t kb0 = c >> 4;            // first block of the lane octet's 4-block group (lanes 8j)
+        const uint32_t code_bytes = min(QCHUNK, (int)(K - c0)) / 2;    // one row's codes in this chunk
+        const uint32_t wcol = (c0 >> 4) + 4 * (lane & 3);          // fan-out: first scale column of word lane % 4
+        int fan_slot = 0;
+        for (int it = 0; it < n_iter; ++it) {
+            const int st = it % QSTAGES;
+            const uint32_t ph = (uint32_t)(it / QSTAGES) & 1u;
+            bool ok = true;
+            if (lane == 0) ok = qwait(ptx::smem_u32(&full_bar[st]), ph, abort_flag, p.dev_status);
+            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
+            const uint8_t *tile = qsm + st * QTILE + warp * QPITCH + lane * 16;
+            const uint32_t rt = r0 + (uint32_t)it * QROWS + (uint32_t)warp;   // this warp's first row of the tile
+            if (fanout) {
+#pragma unroll
+                for (int i = 0; i < QRPW; ++i) {
+                    const uint32_t r = rt + (uint32_t)(i * QWORKERS);
+                    if (lane < fanout) fdst[warp][i][lane] = r < r1 ? p.dst_rows[(int64_t)r * fanout + lane] : -1;
+                }
+                __syncwarp();
+            }
+#pragma unroll
+            for (int i = 0; i < QRPW; ++i) {
+                const uint32_t r = rt + (uint32_t)(i * QWORKERS);
+                if (r >= r1) break;                                   // warp-uniform
+                const uint4 u = active ? *reinterpret_cast<const uint4 *>(tile + i * QWORKERS * QPITCH)
+                                       : make_uint4(0u, 0u, 0u, 0u);
+                const float2 v[4] = {bf16x2_to_f2(u.x), bf16x2_to_f2(u.y), bf16x2_to_f2(u.z), bf16x2_to_f2(u.w)};
+                float m = fmaxf(fmaxf(fmaxf(fabsf(v[0].x), fabsf(v[0].y)), fmaxf(fabsf(v[1].x), fabsf(v[1].y))),
+                                fmaxf(fmaxf(fabsf(v[2].x), fabsf(v[2].y)), fmaxf(fabsf(v[3].x), fabsf(v[3].y))));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                const uint32_t sf_code = block_scale_code(m, s_t, r6);
+                const float4 bt = btab[sf_code];
+                const BlockConst b{bt.x, bt.y, bt.z, __float_as_uint(bt.w)};
+                const uint32_t cw = element_codes8(v, b);
+                if (SCORE || QDQ) {
+                    float2 xh[4];
+                    dequant8(cw, b.sf_h2, s_t, xh);
+                    if (SCORE) {
+                        float2 R[4];
+                        residual8(v, xh, R);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) acc32[k] = fma2(R[k], R[k], acc32[k]);
+                    }
+                    if (QDQ && active) {
+                        uint4 o;
+                        __nv_bfloat162 h;
+                        h = __floats2bfloat162_rn(xh[0].x, xh[0].y); o.x = *reinterpret_cast<uint32_t *>(&h);
+                        h = __floats2bfloat162_rn(xh[1].x, xh[1].y); o.y = *reinterpret_cast<uint32_t *>(&h);
+                        h = __floats2bfloat162_rn(xh[2].x, xh[2].y); o.z = *reinterpret_cast<uint32_t *>(&h);
+                        h = __floats2bfloat162_rn(xh[3].x, xh[3].y); o.w = *reinterpret_cast<uint32_t *>(&h);
+                        *reinterpret_cast<uint4 *>(qdq + r * K + c) = o;
+                    }
+                }
+                if (!codes) continue;
+                // the 4 scale codes of blocks kb0..kb0+3 on lanes 8j
+                uint32_t sw = sf_code | (__shfl_down_sync(0xffffffffu, sf_code, 2) << 8);
+                sw |= __shfl_down_sync(0xffffffffu, sw, 4) << 16;
+                if (!fanout) {
+                    if (active) {
+                        *reinterpret_cast<uint32_t *>(codes + r * (K >> 1) + (c >> 1)) = cw;
+                        if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(scales + sf_off32(r, kb0, K)) = sw;
+                    }
+                    continue;
+                }
+                // fan-out: stage the row's codes, one bulk copy per destination
+                uint32_t *slot = fstage[warp][fan_slot];
+                if (lane < fanout) ptx::bulk_wait_read<QFAN_SLOTS - 1>();
+                __syncwarp();
+                slot[lane] = cw;
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane < fanout) {
+                    const int32_t dst = fdst[warp][i][lane];
+                    if (dst >= 0 && (uint32_t)dst < M_out)
+                        ptx::bulk_store(codes + (uint64_t)dst * (K >> 1) + (c0 >> 1), ptx::smem_u32(slot), code_bytes);
+                    ptx::bulk_commit();
+                }
+                fan_slot = (fan_slot + 1) % QFAN_SLOTS;
+                // scale words: lane l writes word l % 4 of destination l / 4 (+ 8 per round)
+                const uint32_t word = __shfl_sync(0xffffffffu, sw, (lane & 3) * 8);
+                for (int d = lane >> 2; d < fanout; d += 8) {
+                    const int32_t dst = fdst[warp][i][d];
+                    if (dst >= 0 && (uint32_t)dst < M_out && wcol < (K >> 4))
+                        *reinterpret_cast<uint32_t *>(scales + sf_off32((uint32_t)dst, wcol, K)) = word;
+                }
+            }
+            if (SCORE) {
+                // at most QRPW = 4 rows were summed in binary32
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    acc64[2 * k] += (double)acc32[k].x;
+                    acc64[2 * k + 1] += (double)acc32[k].y;
+                    acc32[k] = make_float2(0.0f, 0.0f);
+                }
             }
             __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty_bar[st]));
         }
-#pragma unroll
-        for (int i = 0; i < QROWS / (QTHREADS / 32); ++i) {
-            const int lr = warp + i * (QTHREADS / 32);            // row inside the tile
-            const int64_t r = rt + lr;
-            if (r >= r1) break;                                   // warp-uniform
-            const uint4 u = active ? *reinterpret_cast<const uint4 *>(tile + lr * pitch + lane * 16)
-                                   : make_uint4(0u, 0u, 0u, 0u);
-            float2 v[4] = {bf16x2_to_f2(u.x), bf16x2_to_f2(u.y), bf16x2_to_f2(u.z), bf16x2_to_f2(u.w)};
-            float m = fmaxf(fmaxf(fmaxf(fabsf(v[0].x), fabsf(v[0].y)), fmaxf(fabsf(v[1].x), fabsf(v[1].y))),
-                            fmaxf(fmaxf(fabsf(v[2].x), fabsf(v[2].y)), fmaxf(fabsf(v[3].x), fabsf(v[3].y))));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            const uint32_t sf_code = block_scale_code(m, s_t, r6);
-            const float4 bt = btab[sf_code];
-            const BlockConst b{bt.x, bt.y, bt.z, __float_as_uint(bt.w)};
-            const uint32_t cw = element_codes8(v, b);
-            if (SCORE || QDQ) {
-                float2 xh[4];
-                dequant8(cw, b.sf_h2, s_t, xh);
-                if (SCORE) {
-                    float2 R[4];
-                    residual8(v, xh, R);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) acc32[k] = fma2(R[k], R[k], acc32[k]);
-                }
-                if (QDQ && active) {
-                    uint4 o;
-                    __nv_bfloat162 h;
-                    h = __floats2bfloat162_rn(xh[0].x, xh[0].y); o.x = *reinterpret_cast<uint32_t *>(&h);
-                    h = __floats2bfloat162_rn(xh[1].x, xh[1].y); o.y = *reinterpret_cast<uint32_t *>(&h);
-                    h = __floats2bfloat162_rn(xh[2].x, xh[2].y); o.z = *reinterpret_cast<uint32_t *>(&h);
-                    h = __floats2bfloat162_rn(xh[3].x, xh[3].y); o.w = *reinterpret_cast<uint32_t *>(&h);
-                    *reinterpret_cast<uint4 *>(qdq + r * K + c) = o;
-                }
-            }
-            if (!codes) continue;
-            // the 4 scale codes of blocks kb0..kb0+3 on lanes 8j
-            uint32_t sw = sf_code | (__shfl_down_sync(0xffffffffu, sf_code, 2) << 8);
-            sw |= __shfl_down_sync(0xffffffffu, sw, 4) << 16;
-            if (!fanout) {
-                if (active) {
-                    *reinterpret_cast<uint32_t *>(codes + r * (K >> 1) + (c >> 1)) = cw;
-                    if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(scales + sf_offset(r, kb0, K)) = sw;
-                }
-                continue;
-            }
-            // fan-out: stage the row's codes, one bulk copy per destination
-            uint32_t *slot = fstage[warp][fan_slot];
-            if (lane < fanout) ptx::bulk_wait_read<QFAN_SLOTS - 1>();
-            __syncwarp();
-            slot[lane] = cw;
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane < fanout) {
-                const int64_t dst = fdst[warp][i][lane];
-                if (dst >= 0 && dst < p.M_out) {
-                    ptx::bulk_store(codes + dst * (K >> 1) + (c0 >> 1), ptx::smem_u32(slot), code_bytes);
-                }
-                ptx::bulk_commit();
-            }
-            fan_slot = (fan_slot + 1) % QFAN_SLOTS;
-            // scale words: lane l writes word l % 4 of destination l / 4 (+ 8 per round)
-            const uint32_t word = __shfl_sync(0xffffffffu, sw, (lane & 3) * 8);
-            const int64_t col = (c0 >> 4) + 4 * (lane & 3);       // first scale column of the word
-            for (int d = lane >> 2; d < fanout; d += 8) {
-                const int64_t dst = fdst[warp][i][d];
-                if (dst >= 0 && dst < p.M_out && col < (K >> 4))
-                    *reinterpret_cast<uint32_t *>(scales + sf_offset(dst, col, K)) = word;
-            }
-        }
-        if (SCORE) {
-            // at most QROWS / 8 = 4 rows were summed in binary32
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                acc64[2 * k] += (double)acc32[k].x;
-                acc64[2 * k + 1] += (double)acc32[k].y;
-                acc32[k] = make_float2(0.0f, 0.0f);
-            }
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty_bar[st]));
-        if (threadIdx.x == 0 && issued < n_iter) {
-            // refill this slot once every warp has consumed it
-            if (!qwait(ptx::smem_u32(&empty_bar[st]), ph, abort_flag, p.dev_status)) break;
-            const uint32_t fb = ptx::smem_u32(&full_bar[st]);
-            ptx::mbar_arrive_expect_tx(fb, tile_bytes);
-            ptx::tma_load_2d(ptx::smem_u32(qsm + st * tile_bytes), &tm_x, (int32_t)c0,
-                             (int32_t)(row_base + r0 + (int64_t)issued * QROWS), fb);
-            ++issued;
-        }
-    }
-    if (fanout && lane < fanout) ptx::bulk_wait_all();            // staged rows read and written
-    if (threadIdx.x == 0) {
-        // after an early exit, let every issued copy land before the CTA ends
-        for (int j = it; j < issued; ++j)
-            qwait(ptx::smem_u32(&full_bar[j % QSTAGES]), (uint32_t)(j / QSTAGES) & 1u, abort_flag, p.dev_status,
-                  true);
+        if (fanout && lane < fanout) ptx::bulk_wait_all();        // staged rows read and written
     }
 
     if (SCORE) {
         __syncthreads();                                          // the stage ring is free: reuse it
-        double *red = reinterpret_cast<double *>(qsm);            // [8 warps][256 channels]
+        double *red = reinterpret_cast<double *>(qsm);            // [8 workers][256 channels]
+        if (warp < QWORKERS) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            red[warp * QCHUNK + lane * 8 + i] = acc64[i] + (double)((i & 1) ? acc32[i >> 1].y : acc32[i >> 1].x);
+            for (int i = 0; i < 8; ++i)
+                red[warp * QCHUNK + lane * 8 + i] = acc64[i] + (double)((i & 1) ? acc32[i >> 1].y : acc32[i >> 1].x);
+        }
         __syncthreads();
-        int64_t ch = c0 + threadIdx.x;
-        if (ch < K) {
+        const uint32_t ch = c0 + threadIdx.x;
+        if (threadIdx.x < QCHUNK && ch < K) {
             double sum = 0.0;
 #pragma unroll
-            for (int w = 0; w < QTHREADS / 32; ++w) sum += red[w * QCHUNK + threadIdx.x];
+            for (int w = 0; w < QWORKERS; ++w) sum += red[w * QCHUNK + threadIdx.x];
             p.partials[(int64_t)blockIdx.y * K + ch] = sum;
         }
     }
@@ -691,14 +703,18 @@ static nvfp4_status launch_quantize_t(const CUtensorMap &tm, const QuantParams &
 static nvfp4_status launch_quantize(bool score, const void *x, int64_t rows_total, const void *fallback,
                                     QuantParams &p, dim3 grid, cudaStream_t st)
 {
-    p.box_inner = (int)std::min<int64_t>(QCHUNK, p.K);
+    // every tile row is 256 channels (512 bytes): the box reads zeros past K
+    p.box_inner = QCHUNK;
+    NVFP4_REQUIRE((int64_t)std::max<int64_t>(p.M_out, p.M) * (p.K / 2) < (1ll << 31) &&
+                      (int64_t)p.M * p.K < (1ll << 31),
+                  NVFP4_ERR_UNSUPPORTED_SHAPE, "k_quantize: rows x K must stay below 2^31 elements per tensor");
     CUtensorMap tm;
     const bool empty = rows_total <= 0 || x == nullptr;
     if (!make_tmap_2d(&tm, empty ? fallback : x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)p.K,
                       (uint64_t)(empty ? 1 : rows_total), (uint64_t)p.ldx * 2, (uint32_t)p.box_inner, QROWS,
                       CU_TENSOR_MAP_SWIZZLE_NONE))
         return set_error(NVFP4_ERR_CUDA, "k_quantize: tensor map encoding failed");
-    const size_t smem = (size_t)QSTAGES * QROWS * p.box_inner * 2;
+    const size_t smem = QSMEM;
     if (p.qdq) return launch_quantize_t<false, true>(tm, p, grid, smem, st);
     if (score) return launch_quantize_t<true, false>(tm, p, grid, smem, st);
     return launch_quantize_t<false, false>(tm, p, grid, smem, st);

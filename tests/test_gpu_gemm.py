@@ -175,3 +175,36 @@ def test_gemm_no_routed_rows(cuda, align):
                           epilogue=api.EPI_STORE_F32, row_token=r.row_token, row_gate=r.row_gate, out=out16)
     torch.cuda.synchronize()
     assert torch.all(out == 7.0) and torch.all(y == 3.0) and torch.all(out16 == 5.0)
+
+
+def test_bounded_wait_expiry_reports_timeout(cuda):
+    """A device-side wait that runs out: the test hook withholds the
+    accumulator-ready signal of a one-tile GEMM (1-SM shape) with every wait
+    bounded by 20 ms.  The status word must read NVFP4_ERR_TIMEOUT, the call
+    must return, and the same process must then run the normal GEMM on the
+    same inputs to the oracle's result."""
+    rng = np.random.default_rng(41)
+    T, E, kr, N, K = 128, 1, 1, 256, 256
+    x, w, logits, r, xq, s_w, c_w, sf_w, w_sel, rac_ld = _setup(cuda, rng, T, E, kr, N, K, 0)
+    out = torch.zeros(r.m_pad_max, N, dtype=torch.float32, device=cuda)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda)
+    lib = api._lib.load()
+    api.check(lib.nvfp4_debug_gemm_wait_expiry(
+        api._p(xq.codes), api._p(xq.scales), api._p(xq.s_t), r.m_pad_max, api._p(c_w), api._p(sf_w), api._p(s_w),
+        N, K, E, api._p(r.offsets), api.EPI_STORE_F32, api._p(r.row_token), api._p(r.row_gate), api._p(out), N,
+        api._p(status), 20_000_000, api._stream(cuda)))
+    torch.cuda.synchronize()
+    assert api.read_status(status) == 5, "expected NVFP4_ERR_TIMEOUT"
+    # the context is intact: the normal call on the same inputs is exact
+    status.zero_()
+    api.grouped_gemm(xq.codes, xq.scales, xq.s_t, r.m_pad_max, c_w, sf_w, s_w, N, K, E, r.offsets,
+                     epilogue=api.EPI_STORE_F32, row_token=r.row_token, row_gate=r.row_gate, out=out,
+                     dev_status=status)
+    torch.cuda.synchronize()
+    assert api.read_status(status) == 0
+    qx = oracle.quantize(x)
+    want = qx.xhat.astype(np.float64) @ oracle.quantize(w[0]).xhat.astype(np.float64).T
+    tok = r.row_token.cpu().numpy()[: r.m_pad_max]
+    got = out.cpu().numpy()
+    rows = np.nonzero(tok >= 0)[0]
+    assert rel_fro(got[rows], want[tok[rows]]) <= TOL
