@@ -86,6 +86,9 @@ def _L():
         lib.oracle_rac_residual.argtypes = [F32P, I64, I64, ctypes.c_float, I32P, I64, U16P]
         lib.oracle_route.argtypes = [F32P, I64, I64, I64, I32P, F64P]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_fp8_scale_from_amax.argtypes = [ctypes.c_float]
+        lib.oracle_fp8_scale_from_amax.restype = ctypes.c_float
+        lib.oracle_fp8_quantize.argtypes = [U16P, I64, I64, I64, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
         _lib = lib
     return _lib
 
@@ -302,6 +305,22 @@ def w4a4_rac_matmul(xhat: np.ndarray, s_a: float, rho: np.ndarray | None, S: np.
         r = bf16_to_f32(rho[:, :len(S)]).astype(np.float64) * float(s_a)
         Y += r @ what[:, S].astype(np.float64).T
     return Y
+
+
+def fp8_quantize(x: np.ndarray, s: float | None = None):
+    """Per-tensor FP8 E4M3 quantization of a bf16 matrix (the FP8 rollout the
+    pages compare NVFP4 against, gist.science/it sections 1 and 4; READING:
+    s = max|x| / 448, q = E4M3(fl(x / s)), xhat = fl(e4m3(q) * s)).
+    Returns (codes uint8 [M, K] with the sign in bit 7, xhat float32, s)."""
+    x = np.ascontiguousarray(x, np.uint16)
+    M, K = x.shape
+    if s is None:
+        s = float(_L().oracle_fp8_scale_from_amax(ctypes.c_float(amax(x))))
+    codes = np.empty((M, K), np.uint8)
+    xhat = np.empty((M, K), np.float32)
+    if M:
+        _L().oracle_fp8_quantize(x, M, K, K, ctypes.c_float(s), _ptr(codes), _ptr(xhat))
+    return codes, xhat, float(np.float32(s))
 
 
 def silu(z: np.ndarray) -> np.ndarray:

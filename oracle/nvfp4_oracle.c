@@ -312,6 +312,39 @@ void oracle_route(const float *logits, int64_t T, int64_t E, int64_t kr,
     }
 }
 
+/* ---------------------------------------------------- FP8 (comparison) */
+
+/*
+ * Per-tensor FP8 E4M3 quantization, the format of the FP8 rollout the pages
+ * compare against (gist.science/it, sections 1 and 4: the stable FP8
+ * baseline; NVFP4 GEMMs are quoted at ~2x its throughput).  READING: the
+ * pages give no FP8 recipe; the plainest one is a per-tensor scale that maps
+ * the tensor maximum to E4M3's largest magnitude:
+ *   s = A / 448 (1 when A == 0);  q = E4M3(fl(x / s)) with the sign of x,
+ *   nearest even, saturating at 448;  xhat = fl(e4m3(q) * s).
+ * codes [M x K] (sign in bit 7), xhat [M x K] (either may be NULL).
+ */
+float oracle_fp8_scale_from_amax(float A)
+{
+    if (A == 0.0f) return 1.0f;
+    return A / 448.0f;
+}
+
+void oracle_fp8_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, float s,
+                         uint8_t *codes, float *xhat)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t c = 0; c < K; ++c) {
+            float v = oracle_bf16_to_f32(x[r * ldx + c]);
+            float y = v / s;
+            uint8_t q = oracle_e4m3_encode(fabsf(y));
+            if (signbit(y)) q |= 0x80;
+            if (codes) codes[r * K + c] = q;
+            if (xhat) xhat[r * K + c] = (float)oracle_e4m3_decode(q) * s;
+        }
+}
+
 /* Number of OpenMP threads the oracle runs with (1 without OpenMP). */
 int oracle_num_threads(void)
 {

@@ -100,3 +100,16 @@ def quantize_block_exact(x_bits, s_t_bits):
         xhat.append(xh)
         R.append(rn32(x - xh))
     return sf_code, codes, xhat, R
+
+
+def fp8_quantize_exact(x_bits, s_bits):
+    """Per-tensor E4M3 quantization with one rounding per operation:
+    q = E4M3(fl(x / s)) (sign of x), xhat = fl(e4m3(q) * s)."""
+    s = f32_bits_to_fraction(s_bits)
+    out = []
+    for b in x_bits:
+        x = bf16_bits_to_fraction(b)
+        y = rn32(x / s)
+        c = e4m3_code(abs(y)) | (0x80 if b & 0x8000 else 0)
+        out.append((c, rn32((-1 if c & 0x80 else 1) * E4M3_VAL[c & 0x7F] * s)))
+    return out
