@@ -86,6 +86,8 @@ def _L():
         lib.oracle_rac_residual.argtypes = [F32P, I64, I64, ctypes.c_float, I32P, I64, U16P]
         lib.oracle_route.argtypes = [F32P, I64, I64, I64, I32P, F64P]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_quantize_f32.argtypes = [F32P, I64, I64, I64, ctypes.c_float,
+                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_fp8_scale_from_amax.argtypes = [ctypes.c_float]
         lib.oracle_fp8_scale_from_amax.restype = ctypes.c_float
         lib.oracle_fp8_quantize.argtypes = [U16P, I64, I64, I64, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
@@ -263,6 +265,48 @@ def rac_residual(resid: np.ndarray, s_t: float, S: np.ndarray, k_pad: int | None
     if k_pad is not None and k_pad > k:
         rho = np.concatenate([rho, np.zeros((M, k_pad - k), np.uint16)], axis=1)
     return rho
+
+
+def quantize_f32(x: np.ndarray, s_t: float | None = None) -> Quantized:
+    """NVFP4 quantization of a binary32 matrix with the block steps of
+    quantize(); s_t defaults to max|x| / 2688."""
+    x = np.ascontiguousarray(x, np.float32)
+    M, K = x.shape
+    assert K % 16 == 0
+    if s_t is None:
+        s_t = tensor_scale(float(np.abs(x).max()) if x.size else 0.0)
+    codes = np.empty((M, K // 2), np.uint8)
+    sf = np.empty((M, K // 16), np.uint8)
+    xhat = np.empty((M, K), np.float32)
+    resid = np.empty((M, K), np.float32)
+    if M:
+        _L().oracle_quantize_f32(x, M, K, K, ctypes.c_float(s_t), _ptr(codes), _ptr(sf), _ptr(xhat), _ptr(resid))
+    return Quantized(codes, sf, xhat, resid, float(np.float32(s_t)))
+
+
+def rac_residual_nvfp4(resid: np.ndarray, s_t: float, S: np.ndarray, k_pad: int | None = None):
+    """RAC with the "second pass of quantization" of the selected channels
+    (gist.science/it 2.2 B): the residual R[:, S] (binary32, channels in
+    ascending order) is quantized again to NVFP4 as one [M x k] tensor with
+    its own tensor scale s_r = max|R_S| / 2688 and 16-element blocks along the
+    selected channels (a last partial block zero-padded); the correction uses
+    its dequantized value rhat, carried like the plain residual:
+    rho2[r, j] = bf16(fl(rhat[r, j] / s_t)).  READING: the pages name the
+    second pass but not its format; the block steps are those of quantize().
+    Returns (rho2 bf16 bits [M, k or k_pad], s_r)."""
+    resid = np.ascontiguousarray(resid, np.float32)
+    S = np.ascontiguousarray(S, np.int32)
+    M, k = resid.shape[0], S.size
+    kb = -(-k // 16) * 16
+    RS = np.zeros((M, kb), np.float32)
+    RS[:, :k] = resid[:, S]
+    A = float(np.abs(RS).max()) if RS.size else 0.0
+    q = quantize_f32(RS, tensor_scale(A)) if M and kb else None
+    rhat = q.xhat[:, :k] if q is not None else np.zeros((M, k), np.float32)
+    rho = f32_to_bf16((rhat / np.float32(s_t)).astype(np.float32)) if k else np.zeros((M, 0), np.uint16)
+    if k_pad is not None and k_pad > k:
+        rho = np.concatenate([rho, np.zeros((M, k_pad - k), np.uint16)], axis=1)
+    return rho, (q.s_t if q is not None else 1.0)
 
 
 def qdq(w: np.ndarray):

@@ -22,8 +22,15 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import (quantize, select_topk, channel_score, rac_residual, route,
+from . import (quantize, select_topk, channel_score, rac_residual, rac_residual_nvfp4, route,
                w4a4_rac_matmul, swiglu, f32_to_bf16, bf16_to_f32)
+
+
+def _rac_operand(resid, s_t, S, rac_mode):
+    """RAC residual operand: bf16 residual (default) or the NVFP4 second pass."""
+    if rac_mode == "nvfp4":
+        return rac_residual_nvfp4(resid, s_t, S)[0]
+    return rac_residual(resid, s_t, S)
 
 
 def quantize_weights(w: np.ndarray):
@@ -48,14 +55,14 @@ def gate_up(xq, rho_x, S_x, idx, w13q, inter):
     return h, f32_to_bf16(h.astype(np.float32))
 
 
-def down(h_bf16, idx, gate, w2q, k_h, row_valid=None):
+def down(h_bf16, idx, gate, w2q, k_h, row_valid=None, rac_mode="bf16"):
     """Quantize the routed h rows as one tensor, select S_h, run the down GEMM
     with RAC and combine with the router weights.
     Returns dict(Y [T, H] f64, hq, S_h, rho_h, y2 [T*kr, H])."""
     T, kr = idx.shape
     hq = quantize(h_bf16)
     S_h = select_topk(channel_score(hq.resid, row_valid), k_h)
-    rho_h = rac_residual(hq.resid, hq.s_t, S_h)
+    rho_h = _rac_operand(hq.resid, hq.s_t, S_h, rac_mode)
     H = w2q[0].xhat.shape[0]
     y2 = np.zeros((T * kr, H), np.float64)
     experts = idx.reshape(-1)
@@ -66,15 +73,17 @@ def down(h_bf16, idx, gate, w2q, k_h, row_valid=None):
     return dict(Y=Y, hq=hq, S_h=S_h, rho_h=rho_h, y2=y2)
 
 
-def layer(x, logits, w13q, w2q, kr, k_x, k_h):
-    """Full layer from bf16 X and router logits; weights already quantized."""
+def layer(x, logits, w13q, w2q, kr, k_x, k_h, rac_mode="bf16"):
+    """Full layer from bf16 X and router logits; weights already quantized.
+    rac_mode "nvfp4" takes the RAC operand from the second NVFP4 pass over
+    the selected residual channels (oracle.rac_residual_nvfp4)."""
     idx, gate = route(logits, kr)
     xq = quantize(x)
     S_x = select_topk(channel_score(xq.resid), k_x)
-    rho_x = rac_residual(xq.resid, xq.s_t, S_x)
+    rho_x = _rac_operand(xq.resid, xq.s_t, S_x, rac_mode)
     inter = w13q[0].xhat.shape[0] // 2
     h64, hb = gate_up(xq, rho_x, S_x, idx, w13q, inter)
-    out = down(hb, idx, gate, w2q, k_h)
+    out = down(hb, idx, gate, w2q, k_h, rac_mode=rac_mode)
     out.update(idx=idx, gate=gate, xq=xq, S_x=S_x, rho_x=rho_x, h64=h64, h_bf16=hb)
     return out
 

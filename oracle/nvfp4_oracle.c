@@ -223,6 +223,34 @@ void oracle_quantize(const uint16_t *x, int64_t M, int64_t K, int64_t ldx, float
 }
 
 /*
+ * The same block quantization of a binary32 matrix (the residuals that the
+ * "second pass of quantization" RAC variant quantizes again).  Outputs as for
+ * oracle_quantize; rows of x are ldx floats apart.
+ */
+void oracle_quantize_f32(const float *x, int64_t M, int64_t K, int64_t ldx, float s_t,
+                         uint8_t *codes, uint8_t *sf, float *xhat, float *resid)
+{
+    int64_t nkb = K / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t b = 0; b < nkb; ++b) {
+            float xb[16], xh[16];
+            uint8_t q[16];
+            for (int i = 0; i < 16; ++i) xb[i] = x[r * ldx + b * 16 + i];
+            uint8_t sc = quantize_block(xb, s_t, q, xh);
+            if (sf) sf[r * nkb + b] = sc;
+            if (codes)
+                for (int i = 0; i < 8; ++i)
+                    codes[r * (K / 2) + b * 8 + i] = (uint8_t)(q[2 * i] | (q[2 * i + 1] << 4));
+            for (int i = 0; i < 16; ++i) {
+                if (xhat) xhat[r * K + b * 16 + i] = xh[i];
+                if (resid) resid[r * K + b * 16 + i] = xb[i] - xh[i];
+            }
+        }
+    }
+}
+
+/*
  * Per-channel residual score: score[c] = sum over rows of R[r,c]^2, with R
  * the binary32 residual of oracle_quantize and the sum in binary64, rows in
  * order.  READING: the pages rank channels by "residual magnitude"

@@ -113,3 +113,23 @@ def fp8_quantize_exact(x_bits, s_bits):
         c = e4m3_code(abs(y)) | (0x80 if b & 0x8000 else 0)
         out.append((c, rn32((-1 if c & 0x80 else 1) * E4M3_VAL[c & 0x7F] * s)))
     return out
+
+
+def quantize_block_exact_f32(x_f32_bits, s_t_bits):
+    """quantize_block_exact for binary32 inputs (bit patterns)."""
+    s_t = f32_bits_to_fraction(s_t_bits)
+    xs = [f32_bits_to_fraction(b) for b in x_f32_bits]
+    neg = [bool(b >> 31) for b in x_f32_bits]
+    a = max(abs(x) for x in xs)
+    v = rn32(rn32(a / 6) / s_t)
+    sf_code = e4m3_code(v)
+    sf = E4M3_VAL[sf_code]
+    d = rn32(sf * s_t)
+    codes, xhat = [], []
+    for x, n in zip(xs, neg):
+        y = rn32(x / d) if d != 0 else Fraction(0)
+        q = e2m1_code(y, n)
+        mag = E2M1_MAG[q & 7]
+        codes.append(q)
+        xhat.append(rn32((-mag if q & 8 else mag) * sf * s_t))
+    return sf_code, codes, xhat
