@@ -99,6 +99,7 @@ def parse():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the trainer-side W4A16 line of the default run")
+    ap.add_argument("--no-formats", action="store_true", help="skip the W4A4 / W8A8 / BF16 grouped-GEMM table")
     return ap.parse_args()
 
 
@@ -334,11 +335,83 @@ def run_ours(args):
         out["w4a16"] = {k: w[k] for k in ("metric", "value", "unit", "ms_per_step", "roofline", "qdq", "e2e")}
         out["w4a16"]["config"] = w["config"]["workload"]
         out["gpu_launches"] += w["gpu_launches"]
+    if not args.no_formats:
+        # the same grouped expert GEMMs on the same layer in other formats:
+        # the pages quote native NVFP4 GEMMs at ~2x FP8 and ~4x BF16
+        if "layer" in locals():
+            del layer
+        torch.cuda.empty_cache()
+        out["gemm_formats"] = run_formats(args, dev)
+        out["gpu_launches"] += out["gemm_formats"].pop("_launches")
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=64)
     if rank == 0:
         print(json.dumps(out), flush=True)
     return out
+
+
+def run_formats(args, dev):
+    """Grouped-GEMM time of the large layer (gate/up + down, same routing and
+    shapes) for NVFP4 W4A4 with and without RAC, per-tensor E4M3 W8A8 and BF16
+    (the trainer-side GEMM on NVFP4 fake-quantized weights), each timed with
+    CUDA events around its two GEMM launches over a few layer steps."""
+    import torch
+    from quantization_nvfp4_quantize_b200 import workloads as wl, api
+    from quantization_nvfp4_quantize_b200 import moe as moe_mod
+    cfg = wl.CONFIGS[WORKLOAD]
+    fl = wl.flops(cfg)
+    x = wl.activations(cfg, args.seed, device=dev)
+    logits = wl.router_logits(cfg, args.seed, device=dev)
+    w13, w2 = wl.weights(cfg, args.seed, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    steps = max(3, min(args.steps, 5))
+    res, launches = {}, 0
+
+    def timed_gemms(layer, names):
+        ev = []
+        saved = {n: getattr(api, n) for n in names}
+
+        def wrap(fn):
+            def w(*a, **k):
+                s_ = torch.cuda.Event(enable_timing=True)
+                e_ = torch.cuda.Event(enable_timing=True)
+                s_.record(stream)
+                o = fn(*a, **k)
+                e_.record(stream)
+                ev.append((s_, e_))
+                return o
+            return w
+        for _ in range(2):
+            layer.forward(x, logits)
+        torch.cuda.synchronize()
+        for n in names:
+            setattr(api, n, wrap(saved[n]))
+        try:
+            for _ in range(steps):
+                layer.forward(x, logits)
+            torch.cuda.synchronize()
+        finally:
+            for n in names:
+                setattr(api, n, saved[n])
+        return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+    for name, make, names, n_launch in (
+            ("w4a4_rac", lambda: moe_mod.MoELayerW4A4(w13, w2, cfg.tokens, cfg.topk, cfg.rac_k), ["grouped_gemm"], 16),
+            ("w4a4", lambda: moe_mod.MoELayerW4A4(w13, w2, cfg.tokens, cfg.topk, 0), ["grouped_gemm"], 10),
+            ("w8a8", lambda: moe_mod.MoELayerW8A8(w13, w2, cfg.tokens, cfg.topk), ["w8a8_grouped_gemm"], 8),
+            ("bf16", lambda: moe_mod.MoELayerW4A16(w13, w2, cfg.tokens, cfg.topk), ["bf16_grouped_gemm"], 6)):
+        layer = make()
+        ms = timed_gemms(layer, names)
+        res[name] = {"gemm_ms_per_step": round(ms, 4), "tflops": round(fl["fp4"] / (ms * 1e-3) / 1e12, 1)}
+        launches += n_launch * (steps + 2)
+        del layer
+        torch.cuda.empty_cache()
+    res["w4a4_over_w8a8"] = round(res["w8a8"]["gemm_ms_per_step"] / res["w4a4"]["gemm_ms_per_step"], 3)
+    res["w4a4_over_bf16"] = round(res["bf16"]["gemm_ms_per_step"] / res["w4a4"]["gemm_ms_per_step"], 3)
+    res["rac_overhead"] = round(res["w4a4_rac"]["gemm_ms_per_step"] / res["w4a4"]["gemm_ms_per_step"] - 1, 4)
+    res["flops"] = "2*M*N*K of both expert GEMMs (no RAC), the same for every format"
+    res["_launches"] = launches
+    return res
 
 
 def time_quantize_kernel(layer, x_in, steps, dev):

@@ -122,7 +122,8 @@ NVFP4_API int nvfp4_num_sms(void);
  *   scales_dev   uint8 swizzled, ceil(M_out/128)*128*K/16 bytes.
  *   score_dev    optional float64 [K]: receives the channel scores.  Required
  *                when rac_k > 0.
- *   rac_k        channels to select, 0 <= rac_k <= min(256, K).
+ *   rac_k        channels to select, 0 <= rac_k <= K (the pages' "top k% of
+ *                channels" is rac_k = k% of K).
  *   rac_ld       row stride (elements) of r_sel, rac_ld >= rac_k,
  *                rac_ld % 64 == 0; columns [rac_k, rac_ld) are written as 0.
  *   sel_dev      int32 [rac_k]: selected channels, ascending.
@@ -180,6 +181,30 @@ NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void *x_dev, int64_t M, int6
                                               double *score_dev, int32_t rac_k, int32_t rac_ld,
                                               int32_t *sel_dev, void *r_sel_dev,
                                               int32_t *dev_status, void *stream);
+
+/* --------------------------------------------------------------------------
+ * nvfp4_rac_residual_nvfp4 -- the RAC variant with a second pass of NVFP4
+ * quantization on the selected channels (gist.science/it 2.2 B).  Given the
+ * channel set S (sel_dev, ascending, from nvfp4_quantize) and the tensor
+ * scale s_t of x, the residuals R[r, S_j] = fl(x - xhat) of the valid rows
+ * are quantized again as one [rows x rac_k] tensor: s_r = max|R_S| / 2688 (1
+ * if all zero), 16-element blocks along j (the last block zero-padded), the
+ * NVFP4 block steps of nvfp4_quantize, dequantized value rhat; the RAC
+ * operand becomes r_sel[dst, j] = bf16(fl(rhat / s_t)) for j < rac_k and 0
+ * for rac_k <= j < rac_ld, written like nvfp4_quantize's r_sel (same
+ * m_valid, dst_rows, fanout, M_out semantics), replacing the plain residual.
+ *   s_r_out_dev  optional float32 [1]: receives s_r.
+ *   workspace    nvfp4_rac_residual_nvfp4_workspace_size() bytes.
+ * rac_ld % 64 == 0, rac_k <= rac_ld; x as for nvfp4_quantize.
+ * -------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_rac_residual_nvfp4_workspace_size(void);
+
+NVFP4_API nvfp4_status nvfp4_rac_residual_nvfp4(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
+                                                const int32_t *m_valid_dev, const float *s_t_dev,
+                                                const int32_t *sel_dev, int32_t rac_k, int32_t rac_ld,
+                                                const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
+                                                void *r_sel_dev, float *s_r_out_dev, void *workspace,
+                                                size_t workspace_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
  * nvfp4_qdq_weights -- trainer-side asymmetric QAT weight fake-quantization
@@ -241,7 +266,7 @@ NVFP4_API nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E, 
  *   w_sel[e, n, j] = 0                                          (k <= j < ld)
  * A selected index outside [0, K) also gives a zero column.
  *   codes_dev  uint8 [E x N x K/2], scales_dev swizzled per expert.
- *   w_sel_dev  bf16 [E x N x ld], ld % 64 == 0, k <= ld.
+ *   w_sel_dev  bf16 [E x N x ld], ld % 64 == 0, k <= ld <= 16384.
  * -------------------------------------------------------------------------- */
 NVFP4_API nvfp4_status nvfp4_gather_weight_channels(const uint8_t *codes_dev, const uint8_t *scales_dev,
                                           int32_t E, int64_t N, int64_t K,
@@ -308,7 +333,8 @@ NVFP4_API nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_d
  *                   256: CTA pairs (2-SM tensor-core tiles, cluster launch)
  *                   compute 256-row x 256-feature tiles.
  *   rac_ld          0 (no RAC) or the row stride of rho / w_sel, % 64 == 0,
- *                   <= 256; rho_dev bf16 [M_pad_max x rac_ld] and
+ *                   <= 16384 (rac_ld / 64 BF16 stages per tile); rho_dev
+ *                   bf16 [M_pad_max x rac_ld] and
  *                   w_sel_dev bf16 [E x N x rac_ld].
  * Shapes: K % 256 == 0, N % 256 == 0 (SWIGLU: I % 128 == 0), M_pad_max a
  * multiple of seg_align, E <= 256; pointers 16-byte aligned.  Persistent
@@ -370,6 +396,45 @@ NVFP4_API nvfp4_status moe_bf16_grouped_gemm(
 NVFP4_API nvfp4_status moe_gather_rows_bf16(const void *x_dev, int64_t T, int64_t K, int64_t ldx,
                                             const int32_t *dst_rows_dev, int32_t fanout, void *out_dev,
                                             int64_t ld_out, int64_t M_out, void *stream);
+
+/* --------------------------------------------------------------------------
+ * fp8_quantize / moe_w8a8_grouped_gemm -- the FP8 comparison path: the pages
+ * compare NVFP4 rollout with a stable FP8 rollout and quote native NVFP4
+ * GEMMs at about twice FP8 throughput (gist.science/it sections 1 and 4);
+ * these two calls give the same grouped expert GEMM on E4M3 operands so that
+ * the ratio can be measured on the same shapes.
+ *
+ * fp8_quantize: per-tensor E4M3 of G bf16 tensors [M x K] (row stride ldx,
+ * group stride M*ldx): s = max|x| / 448 (1 for an all-zero tensor), or
+ * s_in_dev[g] when given, or amax_in_dev[0] / 448 (G == 1); codes =
+ * E4M3(fl(x / s)) with the sign of x in bit 7, nearest even, saturating.
+ *   s_out_dev   float32 [G] (required).
+ *   dst_rows_dev optional int32 [M x fanout] (G == 1): routed copies of each
+ *               row, negative entries or entries >= M_out skipped.
+ *   codes_dev   uint8 [G x M_out x K] (M_out >= M without dst_rows).
+ * K % 16 == 0, ldx % 8 == 0, pointers 16-byte aligned.  workspace:
+ * fp8_quantize_workspace_size(G) bytes unless s_in_dev or amax_in_dev.
+ *
+ * moe_w8a8_grouped_gemm: for every routed row r of expert e,
+ *   y[r,n] = s_a * s_b[e] * sum_k e4m3(a)[r,k] e4m3(b_e)[n,k]
+ * (kind::f8f6f4 MMAs, f32 accumulation in TMEM) with the epilogues of
+ * moe_w4a4_grouped_gemm_rac.  a_codes_dev uint8 [M_pad_max x K] in routed
+ * order, b_codes_dev uint8 [E x N x K], a_s_dev float32 [1], b_s_dev float32
+ * [E].  K % 128 == 0, N % 256 == 0; other shapes and errors as for
+ * moe_w4a4_grouped_gemm_rac.
+ * -------------------------------------------------------------------------- */
+NVFP4_API size_t fp8_quantize_workspace_size(int64_t G);
+
+NVFP4_API nvfp4_status fp8_quantize(const void *x_dev, int64_t G, int64_t M, int64_t K, int64_t ldx,
+                                    const float *s_in_dev, const float *amax_in_dev, float *s_out_dev,
+                                    const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out, uint8_t *codes_dev,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+NVFP4_API nvfp4_status moe_w8a8_grouped_gemm(
+    const uint8_t *a_codes_dev, const float *a_s_dev, int64_t M_pad_max, const uint8_t *b_codes_dev,
+    const float *b_s_dev, int64_t N, int64_t K, int32_t E, const int32_t *offsets_dev, int32_t seg_align,
+    int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev, void *out_dev, int64_t ld_out,
+    float *amax_out_dev, int32_t *dev_status, void *stream);
 
 /* --------------------------------------------------------------------------
  * nvfp4_debug_gemm_wait_expiry -- test hook for the bounded device waits of

@@ -51,6 +51,16 @@ SIGNATURES = {
     "moe_gather_rows_bf16": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int32, c_void_p, c_int64,
                                        c_int64, c_void_p]),
     "nvfp4_debug_encode": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
+    "nvfp4_rac_residual_nvfp4_workspace_size": (c_size_t, []),
+    "nvfp4_rac_residual_nvfp4": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_int32,
+                                           c_int32, c_void_p, c_int32, c_int64, c_void_p, c_void_p, c_void_p,
+                                           c_size_t, c_void_p]),
+    "fp8_quantize_workspace_size": (c_size_t, [c_int64]),
+    "fp8_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_int32, c_int64, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_w8a8_grouped_gemm": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_int64, c_int64, c_int32,
+                                        c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_void_p,
+                                        c_void_p, c_void_p]),
     "nvfp4_debug_gemm_wait_expiry": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
                                                c_int64, c_int64, c_int32, c_void_p, c_int32, c_void_p, c_void_p,
                                                c_void_p, c_int64, c_void_p, c_int64, c_void_p]),

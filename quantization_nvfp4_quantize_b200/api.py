@@ -214,6 +214,58 @@ def gather_rows_bf16(x: torch.Tensor, dst_rows: torch.Tensor, m_out: int, *, out
     return out
 
 
+def rac_residual_nvfp4(x: torch.Tensor, q: "Quantized", rac_k: int, rac_ld: int, *, dst_rows=None, fanout=1,
+                       m_out=None, m_valid=None, s_r_out=None):
+    """nvfp4_rac_residual_nvfp4: replace q.r_sel by the second-pass NVFP4
+    residual operand of the channels q.sel (see the header)."""
+    lib = _lib.load()
+    M, K = x.shape
+    if m_out is None:
+        m_out = M
+    ws = _ws(lib.nvfp4_rac_residual_nvfp4_workspace_size(), x.device)
+    check(lib.nvfp4_rac_residual_nvfp4(_p(x), M, K, x.stride(0), _p(m_valid), _p(q.s_t), _p(q.sel), rac_k, rac_ld,
+                                       _p(dst_rows), fanout, m_out, _p(q.r_sel), _p(s_r_out), _p(ws), ws.numel(),
+                                       _stream(x.device)))
+    return q
+
+
+def fp8_quantize(x: torch.Tensor, *, s: torch.Tensor | None = None, amax: torch.Tensor | None = None,
+                 dst_rows: torch.Tensor | None = None, fanout: int = 1, m_out: int | None = None,
+                 codes: torch.Tensor | None = None, s_out: torch.Tensor | None = None):
+    """fp8_quantize (see the header) on bf16 [M, K] or [G, M, K]: per-tensor
+    E4M3 codes (sign in bit 7).  Returns (codes uint8, s float32 [G])."""
+    lib = _lib.load()
+    assert x.dtype == BF16 and x.stride(-1) == 1
+    x3 = x.unsqueeze(0) if x.dim() == 2 else x
+    G, M, K = x3.shape
+    assert G == 1 or x3.is_contiguous()
+    dev = x.device
+    if m_out is None:
+        m_out = M
+    if codes is None:
+        codes = torch.empty((G, m_out, K) if x.dim() == 3 else (m_out, K), dtype=U8, device=dev)
+    if s_out is None:
+        s_out = torch.empty(G, dtype=F32, device=dev)
+    ws = _ws(lib.fp8_quantize_workspace_size(G), dev)
+    check(lib.fp8_quantize(_p(x3), G, M, K, x3.stride(1), _p(s), _p(amax), _p(s_out), _p(dst_rows), fanout, m_out,
+                           _p(codes), _p(ws), ws.numel(), _stream(dev)))
+    return codes, s_out
+
+
+def w8a8_grouped_gemm(a_codes, a_s, m_pad_max, b_codes, b_s, N, K, E, offsets, *, seg_align=128,
+                      epilogue=EPI_STORE_F32, row_token=None, row_gate=None, out=None, ld_out=None, amax_out=None,
+                      dev_status=None):
+    """moe_w8a8_grouped_gemm (see the header): E4M3 A [m_pad_max x K] in
+    routed order times E4M3 B [E x N x K] with per-tensor scales."""
+    lib = _lib.load()
+    if ld_out is None:
+        ld_out = out.stride(0)
+    check(lib.moe_w8a8_grouped_gemm(_p(a_codes), _p(a_s), m_pad_max, _p(b_codes), _p(b_s), N, K, E, _p(offsets),
+                                    seg_align, epilogue, _p(row_token), _p(row_gate), _p(out), ld_out,
+                                    _p(amax_out), _p(dev_status), _stream(out.device)))
+    return out
+
+
 def debug_encode(v: torch.Tensor):
     """nvfp4_debug_encode: (E2M1 codes, E4M3 codes) of float32 values."""
     lib = _lib.load()

@@ -125,6 +125,7 @@ struct Params {
     int64_t ld_out;
     unsigned int *amax_out;    // SwiGLU: max |h| (float bits), or null
     int l2_hints;              // scatter-add: stream A with evict-first loads, reduce into the output with evict-last
+    int fp8;                   // 1: A and B are E4M3 codes (the FP8 kernel instance: kind::f8f6f4 MMAs, no scale factors)
     uint64_t wait_limit_ns;    // bound of every mbarrier wait
     int debug_withhold_acc;    // test hook: no "accumulator ready" signal for the first tile (1-SM shape)
     int32_t *dev_status;
@@ -190,7 +191,7 @@ __device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __e
 // Scale-atom row of the 2D [bytes/256 x 256] view of a scale buffer.
 __device__ __forceinline__ int32_t sf_row(int64_t byte_off) { return (int32_t)(byte_off >> 8); }
 
-template <int STAGES, bool PAIR, bool STAGING>
+template <int STAGES, bool PAIR, bool STAGING, bool FP8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
            const __grid_constant__ CUtensorMap tm_ra, const __grid_constant__ CUtensorMap tm_rb,
@@ -244,7 +245,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
     const int n_tiles = swiglu ? p.inter / 128 : (int)(p.N / BN);
     const int m_tiles = sh->offsets[E] / G::TILE_M;
     const int total = m_tiles * n_tiles;
-    const int nkb = (int)(p.K / 256);
+    const int nkb = (int)(p.K / (FP8 ? 128 : 256));   // main stages: 128 bytes of K per row
     const int nrk = p.rac_ld / 64;
     const int64_t sf_per_expert = ((p.N + 127) / 128) * 128 * (p.K / 16);
 
@@ -262,7 +263,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
             if (PAIR) ptx::prefetch_tmap(role_a ? &tm_sfa : &tm_sfb);
             if (p.rac_ld > 0) ptx::prefetch_tmap(role_a ? &tm_ra : &tm_rb);
             const uint32_t mult = PAIR ? 2u : 1u;
-            const uint32_t tx_fp4 = mult * (role_a ? (A_BYTES + SFA_BYTES) : (G::B_LOCAL + SFB_BYTES));
+            const uint32_t tx_fp4 = mult * (role_a ? (A_BYTES + (FP8 ? 0u : SFA_BYTES))
+                                                   : (G::B_LOCAL + (FP8 ? 0u : SFB_BYTES)));
             const uint32_t tx_rac = mult * (role_a ? A_BYTES : G::B_LOCAL);
             // the scatter-add GEMM reads each A tile once per group of n-tiles:
             // let those lines leave L2 first so the output band stays resident
@@ -306,23 +308,29 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                         if (role_a && hint_a) {
                             if (fp4) {
                                 ptx::tma_load_2d_pair_hint(ptx::smem_u32(sa), &tm_a, kb * 128, arow, lfb, pol_a);
-                                ptx::tma_load_2d_pair_hint(ptx::smem_u32(ssfa), &tm_sfa, 0, sf_row(sfa_off + kb * 2048),
-                                                           lfb, pol_a);
+                                if (!FP8)
+                                    ptx::tma_load_2d_pair_hint(ptx::smem_u32(ssfa), &tm_sfa, 0,
+                                                               sf_row(sfa_off + kb * 2048), lfb, pol_a);
                             } else {
                                 ptx::tma_load_2d_pair_hint(ptx::smem_u32(sa), &tm_ra, rk * 64, arow, lfb, pol_a);
                             }
                         } else if (role_a) {
                             if (fp4) {
                                 ptx::tma_load_2d_pair(ptx::smem_u32(sa), &tm_a, kb * 128, arow, lfb);
-                                ptx::tma_load_2d_pair(ptx::smem_u32(ssfa), &tm_sfa, 0, sf_row(sfa_off + kb * 2048), lfb);
+                                if (!FP8)
+                                    ptx::tma_load_2d_pair(ptx::smem_u32(ssfa), &tm_sfa, 0, sf_row(sfa_off + kb * 2048),
+                                                          lfb);
                             } else {
                                 ptx::tma_load_2d_pair(ptx::smem_u32(sa), &tm_ra, rk * 64, arow, lfb);
                             }
                         } else if (fp4) {
                             ptx::tma_load_2d_pair(ptx::smem_u32(sb), &tm_b, kb * 128, browr, lfb);
-                            ptx::tma_load_2d_pair(ptx::smem_u32(ssfb), &tm_sfb, 0, sf_row(sfb_off0 + kb * 2048), lfb);
-                            ptx::tma_load_2d_pair(ptx::smem_u32(ssfb + SFB_BYTES / 2), &tm_sfb, 0,
-                                                  sf_row(sfb_off1 + kb * 2048), lfb);
+                            if (!FP8) {
+                                ptx::tma_load_2d_pair(ptx::smem_u32(ssfb), &tm_sfb, 0, sf_row(sfb_off0 + kb * 2048),
+                                                      lfb);
+                                ptx::tma_load_2d_pair(ptx::smem_u32(ssfb + SFB_BYTES / 2), &tm_sfb, 0,
+                                                      sf_row(sfb_off1 + kb * 2048), lfb);
+                            }
                         } else {
                             ptx::tma_load_2d_pair(ptx::smem_u32(sb), &tm_rb, rk * 64, browr, lfb);
                         }
@@ -330,7 +338,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                         if (fp4) {
                             if (hint_a) ptx::tma_load_2d_hint(ptx::smem_u32(sa), &tm_a, kb * 128, m0, fb, pol_a);
                             else ptx::tma_load_2d(ptx::smem_u32(sa), &tm_a, kb * 128, m0, fb);
-                            ptx::bulk_load(ptx::smem_u32(ssfa), p.a_scales + sfa_off + kb * 2048, SFA_BYTES, fb);
+                            if (!FP8)
+                                ptx::bulk_load(ptx::smem_u32(ssfa), p.a_scales + sfa_off + kb * 2048, SFA_BYTES, fb);
                         } else if (hint_a) {
                             ptx::tma_load_2d_hint(ptx::smem_u32(sa), &tm_ra, rk * 64, m0, fb, pol_a);
                         } else {
@@ -339,9 +348,11 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                     } else if (fp4) {
                         ptx::tma_load_2d(ptx::smem_u32(sb), &tm_b, kb * 128, brow0, fb);
                         ptx::tma_load_2d(ptx::smem_u32(sb + G::B_LOCAL / 2), &tm_b, kb * 128, brow1, fb);
-                        ptx::bulk_load(ptx::smem_u32(ssfb), p.b_scales + sfb_off0 + kb * 2048, SFB_BYTES / 2, fb);
-                        ptx::bulk_load(ptx::smem_u32(ssfb + SFB_BYTES / 2), p.b_scales + sfb_off1 + kb * 2048,
-                                       SFB_BYTES / 2, fb);
+                        if (!FP8) {
+                            ptx::bulk_load(ptx::smem_u32(ssfb), p.b_scales + sfb_off0 + kb * 2048, SFB_BYTES / 2, fb);
+                            ptx::bulk_load(ptx::smem_u32(ssfb + SFB_BYTES / 2), p.b_scales + sfb_off1 + kb * 2048,
+                                           SFB_BYTES / 2, fb);
+                        }
                     } else {
                         ptx::tma_load_2d(ptx::smem_u32(sb), &tm_rb, rk * 64, brow0, fb);
                         ptx::tma_load_2d(ptx::smem_u32(sb + G::B_LOCAL / 2), &tm_rb, rk * 64, brow1, fb);
@@ -369,6 +380,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
         if (lane == 0 && leader) {
             // --------------------------------------------------- MMA issuer
             const uint32_t idesc4 = ptx::idesc_mxf4nvf4(PAIR ? 256 : 128, BN);
+            const uint32_t idesc8 = ptx::idesc_e4m3(PAIR ? 256 : 128, BN);
             const uint32_t idesc16 = ptx::idesc_bf16(PAIR ? 256 : 128, BN);
             uint32_t stage = 0, phase = 0, drain_phase = 0;
             bool ok = true;
@@ -393,14 +405,19 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                     const uint32_t sfa = tmem + SF_COL + SF_STRIDE * stage, sfb = sfa + 16;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
+                        // 32 bytes of K per MMA: 64 FP4 or 32 E4M3 elements
                         uint64_t ad = ptx::make_sdesc(sa + 32 * kk, 16, 1024, 2);
                         uint64_t bd = ptx::make_sdesc(sb + 32 * kk, 16, 1024, 2);
-                        if (PAIR)
+                        if (FP8) {
+                            if (PAIR) ptx::mma_e4m3_pair(tmem + ACC_COL, ad, bd, idesc8, (kb | kk) != 0);
+                            else ptx::mma_e4m3(tmem + ACC_COL, ad, bd, idesc8, (kb | kk) != 0);
+                        } else if (PAIR) {
                             ptx::mma_mxf4nvf4_pair(tmem + ACC_COL, ad, bd, idesc4, sfa + 4 * kk, sfb + 8 * kk,
                                                    (kb | kk) != 0);
-                        else
+                        } else {
                             ptx::mma_mxf4nvf4(tmem + ACC_COL, ad, bd, idesc4, sfa + 4 * kk, sfb + 8 * kk,
                                               (kb | kk) != 0);
+                        }
                     }
                     if (PAIR) ptx::tc_commit_pair_mc(ptx::smem_u32(&sh->empty[stage]), 3);
                     else ptx::tc_commit(ptx::smem_u32(&sh->empty[stage]));
@@ -476,7 +493,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
                         break;
                     }
                     ptx::tc_fence_after();
-                    if (kb < nkb) {
+                    if (kb < nkb && !FP8) {
                         const uint32_t ssfa = ptx::smem_u32(stage_base + stage * G::STAGE) + A_BYTES + G::B_LOCAL;
                         const uint32_t ssfb = ssfa + SFA_BYTES;
                         const uint32_t sfa = tmem + SF_COL + SF_STRIDE * stage, sfb = sfa + 16;
@@ -639,14 +656,14 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUt
 
 // ----------------------------------------------------------------- host side
 
-template <int STAGES, bool PAIR, bool STAGING>
+template <int STAGES, bool PAIR, bool STAGING, bool FP8>
 static nvfp4_status launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, const CUtensorMap &tm_ra,
                            const CUtensorMap &tm_rb, const CUtensorMap &tm_sfa, const CUtensorMap &tm_sfb,
                            const Params &p, int units, cudaStream_t st)
 {
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
-    auto kern = k_moe_gemm<STAGES, PAIR, STAGING>;
+    auto kern = k_moe_gemm<STAGES, PAIR, STAGING, FP8>;
     const uint32_t smem = Cfg<STAGES, PAIR, STAGING>::SMEM;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return check_launch("k_moe_gemm: device");
@@ -703,13 +720,19 @@ static nvfp4_status dispatch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, c
     if (pair) {
         // 5 stages; the f32 epilogues add their transpose tiles
         const int units = (int)std::min<int64_t>(num_sms() / 2, max_tiles);
-        return swiglu ? launch<5, true, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
-                      : launch<5, true, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
+        if (p.fp8)
+            return swiglu ? launch<5, true, false, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
+                          : launch<5, true, true, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
+        return swiglu ? launch<5, true, false, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
+                      : launch<5, true, true, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
     }
     // SwiGLU (bf16 out): 4 stages; f32 epilogues: 3 stages + transpose tiles
     const int units = (int)std::min<int64_t>(num_sms(), max_tiles);
-    return swiglu ? launch<4, false, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
-                  : launch<3, false, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
+    if (p.fp8)
+        return swiglu ? launch<4, false, false, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
+                      : launch<3, false, true, true>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
+    return swiglu ? launch<4, false, false, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st)
+                  : launch<3, false, true, false>(tm_a, tm_b, tm_ra, tm_rb, tm_sfa, tm_sfb, p, units, st);
 }
 
 }  // namespace gemm
@@ -743,8 +766,8 @@ static nvfp4_status gemm_rac(
                   NVFP4_ERR_UNSUPPORTED_SHAPE,
                   "moe_w4a4_grouped_gemm_rac: M_pad_max must be a positive multiple of seg_align");
     NVFP4_REQUIRE((int64_t)E * N < (1ll << 31), NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_w4a4_grouped_gemm_rac: E*N too large");
-    NVFP4_REQUIRE(rac_ld >= 0 && rac_ld <= 256 && rac_ld % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
-                  "moe_w4a4_grouped_gemm_rac: rac_ld must be 0..256 and a multiple of 64");
+    NVFP4_REQUIRE(rac_ld >= 0 && rac_ld <= 16384 && rac_ld % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "moe_w4a4_grouped_gemm_rac: rac_ld must be 0..16384 and a multiple of 64");
     NVFP4_REQUIRE(rac_ld == 0 || (rho_dev && w_sel_dev), NVFP4_ERR_INVALID_ARG,
                   "moe_w4a4_grouped_gemm_rac: rac_ld > 0 needs rho and w_sel");
     const int inter = (int)(N / 2);
@@ -904,4 +927,68 @@ extern "C" nvfp4_status moe_bf16_grouped_gemm(
     if (p.amax_out && cudaMemsetAsync(p.amax_out, 0, sizeof(float), st) != cudaSuccess)
         return check_launch("moe_bf16_grouped_gemm: memset");
     return dispatch(tm_ra, tm_rb, tm_ra, tm_rb, tm_ra, tm_rb, p, M_pad_max, seg_align, st);
+}
+
+extern "C" nvfp4_status moe_w8a8_grouped_gemm(
+    const uint8_t *a_codes_dev, const float *a_s_dev, int64_t M_pad_max, const uint8_t *b_codes_dev,
+    const float *b_s_dev, int64_t N, int64_t K, int32_t E, const int32_t *offsets_dev, int32_t seg_align,
+    int32_t epilogue, const int32_t *row_token_dev, const float *row_gate_dev, void *out_dev, int64_t ld_out,
+    float *amax_out_dev, int32_t *dev_status, void *stream)
+{
+    using namespace nvfp4::gemm;
+    cudaStream_t st = (cudaStream_t)stream;
+    NVFP4_REQUIRE(a_codes_dev && a_s_dev && b_codes_dev && b_s_dev && offsets_dev && row_token_dev && out_dev,
+                  NVFP4_ERR_INVALID_ARG, "moe_w8a8_grouped_gemm: null pointer");
+    NVFP4_REQUIRE(epilogue >= 0 && epilogue <= 2, NVFP4_ERR_INVALID_ARG, "moe_w8a8_grouped_gemm: bad epilogue");
+    NVFP4_REQUIRE(seg_align == 128 || seg_align == 256, NVFP4_ERR_INVALID_ARG,
+                  "moe_w8a8_grouped_gemm: seg_align must be 128 or 256");
+    NVFP4_REQUIRE(epilogue != MOE_EPI_SCATTER_ADD_F32 || row_gate_dev, NVFP4_ERR_INVALID_ARG,
+                  "moe_w8a8_grouped_gemm: scatter-add needs row_gate");
+    NVFP4_REQUIRE(E >= 1 && E <= MAX_E, NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_w8a8_grouped_gemm: 1 <= E <= 256");
+    NVFP4_REQUIRE(K >= 128 && K % 128 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "moe_w8a8_grouped_gemm: K must be a positive multiple of 128 (K=%lld)", (long long)K);
+    NVFP4_REQUIRE(N >= 256 && N % 256 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "moe_w8a8_grouped_gemm: N must be a positive multiple of 256 (N=%lld)", (long long)N);
+    NVFP4_REQUIRE(M_pad_max >= seg_align && M_pad_max % seg_align == 0 && M_pad_max < (1ll << 31),
+                  NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_w8a8_grouped_gemm: M_pad_max must be a positive multiple of seg_align");
+    NVFP4_REQUIRE((int64_t)E * N < (1ll << 31), NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_w8a8_grouped_gemm: E*N too large");
+    const int inter = (int)(N / 2);
+    if (epilogue == MOE_EPI_SWIGLU_BF16) {
+        NVFP4_REQUIRE(inter % 128 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_w8a8_grouped_gemm: SwiGLU needs I % 128 == 0");
+        NVFP4_REQUIRE(ld_out >= inter && ld_out % 8 == 0, NVFP4_ERR_ALIGNMENT,
+                      "moe_w8a8_grouped_gemm: SwiGLU ld_out must be >= N/2 and a multiple of 8");
+    } else {
+        NVFP4_REQUIRE(ld_out >= N && ld_out % 4 == 0, NVFP4_ERR_ALIGNMENT,
+                      "moe_w8a8_grouped_gemm: ld_out must be >= N and a multiple of 4");
+    }
+    NVFP4_REQUIRE(aligned16(a_codes_dev) && aligned16(b_codes_dev) && aligned16(out_dev), NVFP4_ERR_ALIGNMENT,
+                  "moe_w8a8_grouped_gemm: pointers must be 16-byte aligned");
+    CUtensorMap tm_a, tm_b;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    const bool ok = make_tmap_2d(&tm_a, a_codes_dev, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K, (uint64_t)M_pad_max,
+                                 (uint64_t)K, 128, BOX_ROWS, sw) &&
+                    make_tmap_2d(&tm_b, b_codes_dev, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K, (uint64_t)E * N,
+                                 (uint64_t)K, 128, BOX_ROWS, sw);
+    NVFP4_REQUIRE(ok, NVFP4_ERR_CUDA, "moe_w8a8_grouped_gemm: tensor map encoding failed");
+    Params p{};
+    p.a_s_t = a_s_dev;
+    p.b_s_t = b_s_dev;
+    p.N = N;
+    p.K = K;
+    p.E = E;
+    p.offsets = offsets_dev;
+    p.rac_ld = 0;
+    p.epilogue = epilogue;
+    p.inter = inter;
+    p.row_token = row_token_dev;
+    p.row_gate = row_gate_dev;
+    p.out = out_dev;
+    p.ld_out = ld_out;
+    p.amax_out = (epilogue == MOE_EPI_SWIGLU_BF16) ? reinterpret_cast<unsigned int *>(amax_out_dev) : nullptr;
+    p.wait_limit_ns = TIMEOUT_NS;
+    p.fp8 = 1;
+    p.dev_status = dev_status;
+    if (p.amax_out && cudaMemsetAsync(p.amax_out, 0, sizeof(float), st) != cudaSuccess)
+        return check_launch("moe_w8a8_grouped_gemm: memset");
+    return dispatch(tm_a, tm_b, tm_a, tm_b, tm_a, tm_b, p, M_pad_max, seg_align, st);
 }

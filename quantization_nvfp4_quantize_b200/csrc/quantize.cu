@@ -536,6 +536,84 @@ __global__ void __launch_bounds__(256) k_rac_residual(
     }
 }
 
+// ----------------------------------------- RAC second-pass (NVFP4) variant
+
+// Residual R = fl(x - xhat) of input channel ch of one row (the element's
+// 16-block is re-quantized with the arithmetic of k_quantize).
+__device__ __forceinline__ float residual1(const __nv_bfloat16 *__restrict__ xrow, int64_t ch, float s_t, float2 r6)
+{
+    const __nv_bfloat16 *blk = xrow + (ch & ~15ll);
+    const uint4 u0 = __ldg(reinterpret_cast<const uint4 *>(blk));
+    const uint4 u1 = __ldg(reinterpret_cast<const uint4 *>(blk + 8));
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[i])), fabsf(bf16hi(w[i]))));
+    const BlockConst b = block_const(block_scale_code(m, s_t, r6), s_t);
+    const int idx = (int)(ch & 15);
+    const uint32_t word = w[idx >> 1];
+    const float xv = (idx & 1) ? bf16hi(word) : bf16lo(word);
+    return __fsub_rn(xv, element_xhat1(xv, b, s_t));
+}
+
+// Pass 1: max |R| over the selected channels of the valid rows (one warp per row).
+__global__ void __launch_bounds__(256) k_rac_amax(const __nv_bfloat16 *__restrict__ x, int64_t ldx, int64_t M,
+                                                  const int32_t *__restrict__ m_valid, const float *__restrict__ s_t_ptr,
+                                                  const int32_t *__restrict__ sel, int k, unsigned int *amax_bits)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    int64_t Me = M;
+    if (m_valid) Me = min(Me, (int64_t)max(*m_valid, 0));
+    if (r >= Me) return;
+    const float s_t = *s_t_ptr;
+    const float2 r6 = recip_bracket(__fmul_rn(6.0f, s_t));
+    float m = 0.0f;
+    for (int j = lane; j < k; j += 32) m = fmaxf(m, fabsf(residual1(x + r * ldx, sel[j], s_t, r6)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0 && m > 0.0f) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+// Pass 2: the selected residuals quantized again to NVFP4 as one tensor
+// (scale s_r from pass 1, 16-channel blocks along the selection, the last
+// block zero-padded): rho2 = bf16(fl(rhat / s_t)), written to every
+// destination row.  One warp per row; a half-warp is one block.
+__global__ void __launch_bounds__(256) k_rac_residual_nvfp4(
+    const __nv_bfloat16 *__restrict__ x, int64_t ldx, int64_t M, const int32_t *__restrict__ m_valid,
+    const float *__restrict__ s_t_ptr, const int32_t *__restrict__ sel, int k, int ld,
+    const unsigned int *__restrict__ amax_bits, float *s_r_out, const int32_t *__restrict__ dst_rows, int fanout,
+    int64_t M_out, __nv_bfloat16 *__restrict__ r_sel)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const float s_r = tensor_scale_from_amax(__uint_as_float(*amax_bits));
+    if (r == 0 && lane == 0 && s_r_out) *s_r_out = s_r;
+    int64_t Me = M;
+    if (m_valid) Me = min(Me, (int64_t)max(*m_valid, 0));
+    if (r >= Me) return;
+    const float s_t = *s_t_ptr;
+    const float2 r6 = recip_bracket(__fmul_rn(6.0f, s_t));
+    const float2 r6r = recip_bracket(__fmul_rn(6.0f, s_r));
+    const int nd = dst_rows ? fanout : 1;
+    for (int j0 = 0; j0 < ld; j0 += 32) {
+        const int j = j0 + lane;
+        const float R = j < k ? residual1(x + r * ldx, sel[j], s_t, r6) : 0.0f;
+        float a = fabsf(R);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        const BlockConst b = block_const(block_scale_code(a, s_r, r6r), s_r);
+        const float rhat = element_xhat1(R, b, s_r);
+        const __nv_bfloat16 outv = __float2bfloat16_rn(j < k ? __fdiv_rn(rhat, s_t) : 0.0f);
+        if (j < ld) {
+            for (int d = 0; d < nd; ++d) {
+                const int64_t dst = dst_rows ? (int64_t)dst_rows[r * fanout + d] : r;
+                if (dst >= 0 && dst < M_out) r_sel[dst * ld + j] = outv;
+            }
+        }
+    }
+}
+
 // --------------------------------------------------- weight channel gather
 
 __global__ void k_gather_w_channels(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
@@ -600,29 +678,36 @@ __global__ void k_weights_channel_major(const uint8_t *__restrict__ codes, const
 // bf16) into a shared [channel][feature] tile, then written out transposed as
 // [feature][ld] rows.
 constexpr int GCM_N = 128;                           // output features per CTA
+constexpr int GCM_J = 256;                           // output channels per CTA (blockIdx.z chunks of ld)
 
 __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__restrict__ codes_cm,
                                                               const uint8_t *__restrict__ scales_cm, int64_t N,
                                                               int64_t K, const int32_t *__restrict__ sel, int k,
                                                               int ld, __nv_bfloat16 *__restrict__ out)
 {
-    extern __shared__ float gtile[];                   // [GCM_N features][ld channels]
+    extern __shared__ float gtile[];                   // [GCM_N features][cw channels of this chunk]
     __shared__ float e4[128];                          // E4M3 code -> value (weight scales are non-negative)
-    __shared__ int32_t ssel[256];
+    __shared__ int32_t ssel[GCM_J];
     const int64_t e = blockIdx.y;
     const int64_t n0 = (int64_t)blockIdx.x * GCM_N;
+    // this CTA's chunk of output channels [j0, j0 + cw); out and sel are
+    // addressed through the chunk-local views below
+    const int j0 = blockIdx.z * GCM_J;
+    const int cw = min(GCM_J, ld - j0);
+    const int kc = max(0, min(k - j0, cw));
+    sel += j0;
     if (threadIdx.x < 128) e4[threadIdx.x] = e4m3_to_f32(threadIdx.x);
-    for (int j = threadIdx.x; j < k; j += blockDim.x) ssel[j] = sel[j];
+    for (int j = threadIdx.x; j < kc; j += blockDim.x) ssel[j] = sel[j];
     __syncthreads();
     // phase 1: item (channel j, 32 features): 16 B of codes, 32 B of scales;
     // consecutive threads take consecutive channels, so the 32 shared-memory
     // stores of an item hit 32 consecutive words across the warp
     const int groups = GCM_N / 32;
-    for (int idx = threadIdx.x; idx < ld * groups; idx += blockDim.x) {
-        const int jj = idx % ld;
-        const int f0 = (idx / ld) * 32;
+    for (int idx = threadIdx.x; idx < cw * groups; idx += blockDim.x) {
+        const int jj = idx % cw;
+        const int f0 = (idx / cw) * 32;
         float v[32];
-        const int64_t ch = jj < k ? (int64_t)ssel[jj] : -1;
+        const int64_t ch = jj < kc ? (int64_t)ssel[jj] : -1;
         if (ch >= 0 && ch < K && n0 + f0 < N) {        // channels outside [0, K) give zeros
             const uint4 w = *reinterpret_cast<const uint4 *>(codes_cm + (e * K + ch) * (N / 2) + (n0 + f0) / 2);
             const uint4 *sp = reinterpret_cast<const uint4 *>(scales_cm + (e * (K / 16) + (ch >> 4)) * N + n0 + f0);
@@ -644,24 +729,24 @@ __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__r
             for (int f = 0; f < 32; ++f) v[f] = 0.0f;
         }
 #pragma unroll
-        for (int f = 0; f < 32; ++f) gtile[(f0 + f) * ld + jj] = v[f];
+        for (int f = 0; f < 32; ++f) gtile[(f0 + f) * cw + jj] = v[f];
     }
     __syncthreads();
     // phase 2: 16 B (8 channels) per thread, ld / 8 threads per output row:
     // each row of out[e, n0 + f, :] is written as one contiguous run
-    const int cpr = ld / 8;
+    const int cpr = cw / 8;
     for (int idx = threadIdx.x; idx < GCM_N * cpr; idx += blockDim.x) {
         const int f = idx / cpr;
-        const int j0 = (idx - f * cpr) * 8;
+        const int jc = (idx - f * cpr) * 8;
         if (n0 + f >= N) break;                        // rows are monotone in idx
-        const float4 a = *reinterpret_cast<const float4 *>(gtile + f * ld + j0);
-        const float4 b = *reinterpret_cast<const float4 *>(gtile + f * ld + j0 + 4);
+        const float4 a = *reinterpret_cast<const float4 *>(gtile + f * cw + jc);
+        const float4 b = *reinterpret_cast<const float4 *>(gtile + f * cw + jc + 4);
         uint4 o;
         o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.x)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.y)) << 16);
         o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.z)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.w)) << 16);
         o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.x)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.y)) << 16);
         o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.z)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.w)) << 16);
-        *reinterpret_cast<uint4 *>(out + (e * N + n0 + f) * ld + j0) = o;
+        *reinterpret_cast<uint4 *>(out + (e * N + n0 + f) * ld + j0 + jc) = o;
     }
 }
 
@@ -759,8 +844,7 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
                   "nvfp4_quantize: fanout must be in [1, 32] with dst_rows");
     NVFP4_REQUIRE(dst_rows_dev != nullptr || M_out >= M, NVFP4_ERR_INVALID_ARG,
                   "nvfp4_quantize: M_out must be >= M without dst_rows");
-    NVFP4_REQUIRE(rac_k >= 0 && rac_k <= 256 && rac_k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
-                  "nvfp4_quantize: rac_k must be in [0, min(256, K)]");
+    NVFP4_REQUIRE(rac_k >= 0 && rac_k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize: rac_k must be in [0, K]");
     if (rac_k > 0) {
         NVFP4_REQUIRE(sel_dev && r_sel_dev, NVFP4_ERR_INVALID_ARG,
                       "nvfp4_quantize: rac_k > 0 needs sel and r_sel");
@@ -839,6 +923,43 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
     return NVFP4_OK;
 }
 
+extern "C" size_t nvfp4_rac_residual_nvfp4_workspace_size(void) { return 256; }
+
+extern "C" nvfp4_status nvfp4_rac_residual_nvfp4(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
+                                                 const int32_t *m_valid_dev, const float *s_t_dev,
+                                                 const int32_t *sel_dev, int32_t rac_k, int32_t rac_ld,
+                                                 const int32_t *dst_rows_dev, int32_t fanout, int64_t M_out,
+                                                 void *r_sel_dev, float *s_r_out_dev, void *workspace,
+                                                 size_t workspace_bytes, void *stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    NVFP4_REQUIRE(M >= 0 && K > 0 && M_out >= 0, NVFP4_ERR_INVALID_ARG, "nvfp4_rac_residual_nvfp4: bad sizes");
+    NVFP4_REQUIRE(s_t_dev && (M == 0 || x_dev) && (rac_k == 0 || sel_dev) && r_sel_dev, NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_rac_residual_nvfp4: x, s_t, sel and r_sel are required");
+    NVFP4_REQUIRE(K % 64 == 0 && K <= 16384, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_rac_residual_nvfp4: K must be a multiple of 64 and <= 16384");
+    NVFP4_REQUIRE(ldx >= K && ldx % 8 == 0 && aligned16(x_dev), NVFP4_ERR_ALIGNMENT,
+                  "nvfp4_rac_residual_nvfp4: x must be 16-byte aligned with ldx >= K, ldx % 8 == 0");
+    NVFP4_REQUIRE(rac_k >= 0 && rac_k <= K && rac_ld >= rac_k && rac_ld % 64 == 0 && rac_ld > 0,
+                  NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_rac_residual_nvfp4: need 0 <= rac_k <= rac_ld, rac_ld % 64 == 0");
+    NVFP4_REQUIRE(dst_rows_dev == nullptr || (fanout >= 1 && fanout <= 32), NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_rac_residual_nvfp4: fanout must be in [1, 32] with dst_rows");
+    NVFP4_REQUIRE(workspace && workspace_bytes >= 256 && aligned16(workspace), NVFP4_ERR_WORKSPACE,
+                  "nvfp4_rac_residual_nvfp4: workspace of 256 bytes required");
+    unsigned int *slot = reinterpret_cast<unsigned int *>(workspace);
+    if (cudaMemsetAsync(slot, 0, 4, st) != cudaSuccess) return check_launch("nvfp4_rac_residual_nvfp4: memset");
+    const unsigned blocks = (unsigned)std::max<int64_t>(1, (M + 7) / 8);
+    if (M > 0 && rac_k > 0) {
+        k_rac_amax<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, m_valid_dev, s_t_dev, sel_dev, rac_k,
+                                           slot);
+        if (check_launch("k_rac_amax") != NVFP4_OK) return NVFP4_ERR_CUDA;
+    }
+    k_rac_residual_nvfp4<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, m_valid_dev, s_t_dev, sel_dev,
+                                                 rac_k, rac_ld, slot, s_r_out_dev, dst_rows_dev,
+                                                 dst_rows_dev ? fanout : 1, M_out, (__nv_bfloat16 *)r_sel_dev);
+    return check_launch("k_rac_residual_nvfp4");
+}
+
 extern "C" size_t nvfp4_qdq_workspace_size(int64_t G, int64_t rows, int64_t cols)
 {
     (void)rows; (void)cols;
@@ -904,8 +1025,8 @@ extern "C" nvfp4_status nvfp4_gather_weight_channels(const uint8_t *codes_dev, c
                   "nvfp4_gather_weight_channels: null pointer");
     NVFP4_REQUIRE(E >= 1 && N >= 1 && K >= 64 && K % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
                   "nvfp4_gather_weight_channels: bad shape");
-    NVFP4_REQUIRE(k >= 0 && k <= ld && ld % 64 == 0 && ld <= 256 && k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
-                  "nvfp4_gather_weight_channels: need 0 <= k <= ld <= 256, ld % 64 == 0");
+    NVFP4_REQUIRE(k >= 0 && k <= ld && ld % 64 == 0 && ld <= 16384 && k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_gather_weight_channels: need 0 <= k <= ld <= 16384, ld % 64 == 0");
     int64_t total = (int64_t)E * N * ld;
     int blocks = (int)std::min<int64_t>((int64_t)num_sms() * 16, (total + 255) / 256);
     k_gather_w_channels<<<blocks, 256, 0, st>>>(codes_dev, scales_dev, E, N, K, sel_dev, k, ld,
@@ -936,11 +1057,11 @@ extern "C" nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_
                   "nvfp4_gather_weight_channels_cm: null pointer");
     NVFP4_REQUIRE(E >= 1 && E <= 65535 && N >= 64 && N % 64 == 0 && K >= 64 && K % 64 == 0,
                   NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_gather_weight_channels_cm: need N % 64 == 0, K % 64 == 0");
-    NVFP4_REQUIRE(k >= 0 && k <= ld && ld % 64 == 0 && ld <= 256 && k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
-                  "nvfp4_gather_weight_channels_cm: need 0 <= k <= ld <= 256, ld % 64 == 0");
+    NVFP4_REQUIRE(k >= 0 && k <= ld && ld % 64 == 0 && ld <= 16384 && k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_gather_weight_channels_cm: need 0 <= k <= ld <= 16384, ld % 64 == 0");
     NVFP4_REQUIRE(aligned16(w_sel_dev) && aligned16(codes_cm_dev) && aligned16(scales_cm_dev), NVFP4_ERR_ALIGNMENT,
                   "nvfp4_gather_weight_channels_cm: pointers must be 16-byte aligned");
-    size_t smem = (size_t)ld * GCM_N * sizeof(float);
+    size_t smem = (size_t)std::min(ld, GCM_J) * GCM_N * sizeof(float);
     {
         static std::once_flag once[64];
         static cudaError_t attr_err[64];
@@ -949,16 +1070,136 @@ extern "C" nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_
             return check_launch("nvfp4_gather_weight_channels_cm: device");
         std::call_once(once[dev], [&] {
             attr_err[dev] = cudaFuncSetAttribute(k_gather_w_channels_cm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)(256 * GCM_N * sizeof(float)));
+                                                 (int)(GCM_J * GCM_N * sizeof(float)));
         });
         if (attr_err[dev] != cudaSuccess)
             return set_error(NVFP4_ERR_CUDA, "nvfp4_gather_weight_channels_cm: smem attribute: %s",
                              cudaGetErrorString(attr_err[dev]));
     }
-    dim3 grid((unsigned)((N + GCM_N - 1) / GCM_N), (unsigned)E);
+    dim3 grid((unsigned)((N + GCM_N - 1) / GCM_N), (unsigned)E, (unsigned)((ld + GCM_J - 1) / GCM_J));
     k_gather_w_channels_cm<<<grid, 256, smem, (cudaStream_t)stream>>>(codes_cm_dev, scales_cm_dev, N, K, sel_dev, k,
                                                                     ld, (__nv_bfloat16 *)w_sel_dev);
     return check_launch("k_gather_w_channels_cm");
+}
+
+// ------------------------------------------------ FP8 E4M3 (comparison)
+//
+// Per-tensor E4M3 quantization, the format of the FP8 rollout the QUADS pages
+// compare against: s = A / 448 (1 for an all-zero tensor), q = E4M3(fl(x/s))
+// with the sign of x, nearest even, saturating.  Each decision is taken from
+// the bracketing multiplications (see the NVFP4 block steps in common.cuh),
+// the IEEE division being evaluated when they disagree.  16 elements per
+// thread; G groups (one scale each) or, for G = 1, routed copies.
+
+namespace nvfp4 {
+
+__global__ void __launch_bounds__(256) k_fp8_quantize(const __nv_bfloat16 *__restrict__ x, int64_t ldx, int64_t M,
+                                                      int64_t K, int64_t group_stride, const float *__restrict__ s_in,
+                                                      const unsigned int *__restrict__ amax_bits, float *s_out,
+                                                      const int32_t *__restrict__ dst_rows, int fanout, int64_t M_out,
+                                                      uint8_t *__restrict__ codes, int64_t codes_gstride)
+{
+    const int g = blockIdx.y;
+    float s;
+    if (s_in) {
+        s = s_in[g];
+    } else {
+        const float A = __uint_as_float(amax_bits[g]);
+        s = A == 0.0f ? 1.0f : __fdiv_rn(A, 448.0f);
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0 && s_out) s_out[g] = s;
+    const float2 rb = recip_bracket(s);
+    const __nv_bfloat16 *xg = x + (int64_t)g * group_stride;
+    uint8_t *cg = codes + (int64_t)g * codes_gstride;
+    const int64_t cpr = K / 16;
+    const int64_t total = M * cpr;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / cpr, c = (i - r * cpr) * 16;
+        const uint4 *src = reinterpret_cast<const uint4 *>(xg + r * ldx + c);
+        const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 a = bf16x2_to_f2(w[2 * k]), b = bf16x2_to_f2(w[2 * k + 1]);
+            const float2 al = mul2(a, make_float2(rb.x, rb.x)), ah = mul2(a, make_float2(rb.y, rb.y));
+            const float2 bl = mul2(b, make_float2(rb.x, rb.x)), bh = mul2(b, make_float2(rb.y, rb.y));
+            lo[k] = (cvt_e4m3x2(al.x, al.y) & 0xFFFFu) | (cvt_e4m3x2(bl.x, bl.y) << 16);
+            hi[k] = (cvt_e4m3x2(ah.x, ah.y) & 0xFFFFu) | (cvt_e4m3x2(bh.x, bh.y) << 16);
+        }
+        if (lo[0] != hi[0] || lo[1] != hi[1] || lo[2] != hi[2] || lo[3] != hi[3]) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 a = bf16x2_to_f2(w[2 * k]), b = bf16x2_to_f2(w[2 * k + 1]);
+                lo[k] = (cvt_e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s)) & 0xFFFFu) |
+                        (cvt_e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s)) << 16);
+            }
+        }
+        const uint4 out = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        if (!dst_rows) {
+            *reinterpret_cast<uint4 *>(cg + r * K + c) = out;
+        } else {
+            for (int j = 0; j < fanout; ++j) {
+                const int64_t d = dst_rows[r * fanout + j];
+                if (d >= 0 && d < M_out) *reinterpret_cast<uint4 *>(cg + d * K + c) = out;
+            }
+        }
+    }
+}
+
+}  // namespace nvfp4
+
+extern "C" size_t fp8_quantize_workspace_size(int64_t G)
+{
+    if (G <= 0) return 0;
+    return (size_t)(((G * 4) + 255) / 256 * 256);
+}
+
+extern "C" nvfp4_status fp8_quantize(const void *x_dev, int64_t G, int64_t M, int64_t K, int64_t ldx,
+                                     const float *s_in_dev, const float *amax_in_dev, float *s_out_dev,
+                                     const int32_t *dst_rows_dev,
+                                     int32_t fanout, int64_t M_out, uint8_t *codes_dev, void *workspace,
+                                     size_t workspace_bytes, void *stream)
+{
+    using namespace nvfp4;
+    cudaStream_t st = (cudaStream_t)stream;
+    NVFP4_REQUIRE(G >= 1 && G <= 65535 && M >= 0 && K > 0 && M_out >= 0, NVFP4_ERR_INVALID_ARG, "fp8_quantize: bad sizes");
+    NVFP4_REQUIRE(s_out_dev && (M == 0 || x_dev) && (M_out == 0 || codes_dev), NVFP4_ERR_INVALID_ARG,
+                  "fp8_quantize: x, s_out and codes are required");
+    NVFP4_REQUIRE(K % 16 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "fp8_quantize: K must be a multiple of 16");
+    NVFP4_REQUIRE(ldx >= K && ldx % 8 == 0, NVFP4_ERR_ALIGNMENT, "fp8_quantize: ldx must be >= K and a multiple of 8");
+    NVFP4_REQUIRE(aligned16(x_dev) && aligned16(codes_dev), NVFP4_ERR_ALIGNMENT,
+                  "fp8_quantize: x and codes must be 16-byte aligned");
+    NVFP4_REQUIRE(dst_rows_dev == nullptr || (G == 1 && fanout >= 1 && fanout <= 32), NVFP4_ERR_INVALID_ARG,
+                  "fp8_quantize: dst_rows needs G == 1 and 1 <= fanout <= 32");
+    NVFP4_REQUIRE(dst_rows_dev != nullptr || M_out >= M, NVFP4_ERR_INVALID_ARG,
+                  "fp8_quantize: M_out must be >= M without dst_rows");
+    NVFP4_REQUIRE(amax_in_dev == nullptr || G == 1, NVFP4_ERR_INVALID_ARG, "fp8_quantize: amax_in needs G == 1");
+    const size_t need = fp8_quantize_workspace_size(G);
+    const bool need_amax = !s_in_dev && !amax_in_dev;
+    NVFP4_REQUIRE(!need_amax || (workspace && workspace_bytes >= need && aligned16(workspace)), NVFP4_ERR_WORKSPACE,
+                  "fp8_quantize: workspace of %zu bytes (16-byte aligned) required", need);
+    // non-negative floats order like their bit patterns
+    const unsigned int *amax_bits = amax_in_dev ? reinterpret_cast<const unsigned int *>(amax_in_dev)
+                                                : reinterpret_cast<unsigned int *>(workspace);
+    if (need_amax) {
+        unsigned int *slots = reinterpret_cast<unsigned int *>(workspace);
+        if (cudaMemsetAsync(slots, 0, (size_t)G * 4, st) != cudaSuccess) return check_launch("fp8_quantize: memset");
+        if (M > 0) {
+            const int64_t want = std::max<int64_t>(1, (int64_t)num_sms() * 8 / G);
+            const int blocks = (int)std::min<int64_t>(want, std::max<int64_t>(1, (M * K / 8 + 255) / 256));
+            k_amax<<<dim3(blocks, (unsigned)G), 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, nullptr,
+                                                              M * ldx, slots);
+            if (check_launch("k_amax (fp8)") != NVFP4_OK) return NVFP4_ERR_CUDA;
+        }
+    }
+    const int64_t chunks = M * (K / 16);
+    const int64_t want = std::max<int64_t>(1, (int64_t)num_sms() * 8 / G);
+    const int blocks = (int)std::min<int64_t>(want, std::max<int64_t>(1, (chunks + 255) / 256));
+    k_fp8_quantize<<<dim3(blocks, (unsigned)G), 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, M * ldx,
+                                                              s_in_dev, amax_bits, s_out_dev, dst_rows_dev,
+                                                              dst_rows_dev ? fanout : 1, M_out, codes_dev, M_out * K);
+    return check_launch("k_fp8_quantize");
 }
 
 // ------------------------------------------------------- conversion probe

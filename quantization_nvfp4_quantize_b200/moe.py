@@ -27,17 +27,30 @@ import torch
 from . import api
 
 
+def rac_channels(percent: float, K: int) -> int:
+    """RAC channel count for "the top k% of channels" (gist.science/it 2.2 B,
+    e.g. 50%): round(percent / 100 * K)."""
+    return int(round(percent / 100.0 * K))
+
+
 class MoELayerW4A4:
+    """rac_k: RAC channels of the gate/up input X (and of h unless rac_k_h is
+    given); see rac_channels for a percentage."""
+
     def __init__(self, w13: torch.Tensor, w2: torch.Tensor, tokens: int, topk: int, rac_k: int,
-                 seg_align: int = 256):
+                 seg_align: int = 256, rac_k_h: int | None = None, rac_mode: str = "bf16"):
         assert w13.dtype == torch.bfloat16 and w2.dtype == torch.bfloat16
         E, N13, H = w13.shape
         E2, H2, I = w2.shape
         assert E2 == E and H2 == H and N13 == 2 * I
         dev = w13.device
         self.E, self.H, self.I, self.T, self.k_r = E, H, I, tokens, topk
+        assert rac_mode in ("bf16", "nvfp4")
+        self.rac_mode = rac_mode            # "nvfp4": second NVFP4 pass over the selected residual channels
         self.rac_k = rac_k
+        self.rac_k_h = rac_k if rac_k_h is None else rac_k_h
         self.rac_ld = -(-rac_k // 64) * 64 if rac_k else 0
+        self.rac_ld_h = -(-self.rac_k_h // 64) * 64 if self.rac_k_h else 0
         _, self.s13, self.c13, self.sf13 = api.qdq_weights(w13, want_qdq=False, want_packed=True)
         _, self.s2, self.c2, self.sf2 = api.qdq_weights(w2, want_qdq=False, want_packed=True)
         # channel-major copies: the per-step RAC gathers read only the selected channels
@@ -45,7 +58,7 @@ class MoELayerW4A4:
         self.c2_cm, self.sf2_cm = api.weights_channel_major(self.c2, self.sf2, H, I)
         self.seg_align = seg_align          # 256: 2-SM GEMM tiles; 128: one SM per tile
         self.m_pad = api.padded_rows_bound(tokens, topk, E, seg_align)
-        mp, ld = self.m_pad, max(self.rac_ld, 1)
+        mp, ld, ldh = self.m_pad, max(self.rac_ld, 1), max(self.rac_ld_h, 1)
         self.xq = api.Quantized(
             codes=torch.empty(mp, H // 2, dtype=torch.uint8, device=dev),
             scales=torch.empty(api.scale_bytes(mp, H), dtype=torch.uint8, device=dev),
@@ -58,10 +71,10 @@ class MoELayerW4A4:
             scales=torch.empty(api.scale_bytes(mp, I), dtype=torch.uint8, device=dev),
             s_t=torch.empty(1, dtype=torch.float32, device=dev),
             score=torch.empty(I, dtype=torch.float64, device=dev),
-            sel=torch.empty(max(rac_k, 1), dtype=torch.int32, device=dev),
-            r_sel=torch.empty(mp, ld, dtype=torch.bfloat16, device=dev))
+            sel=torch.empty(max(self.rac_k_h, 1), dtype=torch.int32, device=dev),
+            r_sel=torch.empty(mp, ldh, dtype=torch.bfloat16, device=dev))
         self.w_sel13 = torch.empty(E, 2 * I, ld, dtype=torch.bfloat16, device=dev)
-        self.w_sel2 = torch.empty(E, H, ld, dtype=torch.bfloat16, device=dev)
+        self.w_sel2 = torch.empty(E, H, ldh, dtype=torch.bfloat16, device=dev)
         self.h = torch.empty(mp, I, dtype=torch.bfloat16, device=dev)
         self.y = torch.empty(tokens, H, dtype=torch.float32, device=dev)
         self.h_amax = torch.empty(1, dtype=torch.float32, device=dev)
@@ -71,11 +84,13 @@ class MoELayerW4A4:
         self.routing = None
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor) -> torch.Tensor:
-        E, H, I, k = self.E, self.H, self.I, self.rac_k
+        E, H, I, k, kh = self.E, self.H, self.I, self.rac_k, self.rac_k_h
         r = api.route(logits, self.k_r, self.m_pad, self.seg_align) if self.routing is None else self._route_into(logits)
         self.routing = r
         api.quantize(x, rac_k=k, rac_ld=self.rac_ld, dst_rows=r.dst_row, fanout=self.k_r, m_out=self.m_pad,
                      out=self.xq, workspace=self.ws_x)
+        if k and self.rac_mode == "nvfp4":
+            api.rac_residual_nvfp4(x, self.xq, k, self.rac_ld, dst_rows=r.dst_row, fanout=self.k_r, m_out=self.m_pad)
         if k:
             api.gather_weight_channels_cm(self.c13_cm, self.sf13_cm, 2 * I, H, self.xq.sel, k, self.rac_ld,
                                           out=self.w_sel13)
@@ -83,14 +98,16 @@ class MoELayerW4A4:
                          2 * I, H, E, r.offsets, seg_align=self.seg_align, rac_ld=self.rac_ld if k else 0, rho=self.xq.r_sel,
                          w_sel=self.w_sel13, epilogue=api.EPI_SWIGLU_BF16, row_token=r.row_token,
                          row_gate=r.row_gate, out=self.h, amax_out=self.h_amax)
-        api.quantize(self.h, rac_k=k, rac_ld=self.rac_ld, m_out=self.m_pad, m_valid=r.offsets[E:],
+        api.quantize(self.h, rac_k=kh, rac_ld=self.rac_ld_h, m_out=self.m_pad, m_valid=r.offsets[E:],
                      amax=self.h_amax, out=self.hq, workspace=self.ws_h)
-        if k:
-            api.gather_weight_channels_cm(self.c2_cm, self.sf2_cm, H, I, self.hq.sel, k, self.rac_ld,
+        if kh and self.rac_mode == "nvfp4":
+            api.rac_residual_nvfp4(self.h, self.hq, kh, self.rac_ld_h, m_out=self.m_pad, m_valid=r.offsets[E:])
+        if kh:
+            api.gather_weight_channels_cm(self.c2_cm, self.sf2_cm, H, I, self.hq.sel, kh, self.rac_ld_h,
                                           out=self.w_sel2)
         self.y.zero_()
         api.grouped_gemm(self.hq.codes, self.hq.scales, self.hq.s_t, self.m_pad, self.c2, self.sf2, self.s2,
-                         H, I, E, r.offsets, seg_align=self.seg_align, rac_ld=self.rac_ld if k else 0,
+                         H, I, E, r.offsets, seg_align=self.seg_align, rac_ld=self.rac_ld_h if kh else 0,
                          rho=self.hq.r_sel, w_sel=self.w_sel2,
                          epilogue=api.EPI_SCATTER_ADD_F32, row_token=r.row_token, row_gate=r.row_gate, out=self.y)
         return self.y
@@ -164,6 +181,48 @@ class MoELayerW4A16:
         api.bf16_grouped_gemm(self.h, self.m_pad, self.wq2, H, I, E, r.offsets, seg_align=self.seg_align,
                               epilogue=api.EPI_SCATTER_ADD_F32, row_token=r.row_token, row_gate=r.row_gate,
                               out=self.y)
+        return self.y
+
+    _route_into = MoELayerW4A4._route_into
+
+
+class MoELayerW8A8:
+    """The FP8 rollout the pages compare NVFP4 against (gist.science/it
+    sections 1 and 4), on the same expert layer: per-tensor E4M3 weights
+    (quantized once) and activations (quantized online, X to its routed rows,
+    h with the scale from the gate/up epilogue's max |h|), grouped E4M3 GEMMs
+    with the SwiGLU and router-weighted combine epilogues.  No RAC."""
+
+    def __init__(self, w13: torch.Tensor, w2: torch.Tensor, tokens: int, topk: int, seg_align: int = 256):
+        E, N13, H = w13.shape
+        _, _, I = w2.shape
+        dev = w13.device
+        self.E, self.H, self.I, self.T, self.k_r, self.seg_align = E, H, I, tokens, topk, seg_align
+        self.c13, self.s13 = api.fp8_quantize(w13.contiguous())
+        self.c2, self.s2 = api.fp8_quantize(w2.contiguous())
+        self.m_pad = api.padded_rows_bound(tokens, topk, E, seg_align)
+        self.xc = torch.empty(self.m_pad, H, dtype=torch.uint8, device=dev)
+        self.xs = torch.empty(1, dtype=torch.float32, device=dev)
+        self.h = torch.empty(self.m_pad, I, dtype=torch.bfloat16, device=dev)
+        self.hc = torch.empty(self.m_pad, I, dtype=torch.uint8, device=dev)
+        self.hs = torch.empty(1, dtype=torch.float32, device=dev)
+        self.h_amax = torch.empty(1, dtype=torch.float32, device=dev)
+        self.y = torch.empty(tokens, H, dtype=torch.float32, device=dev)
+        self.routing = None
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor) -> torch.Tensor:
+        E, H, I = self.E, self.H, self.I
+        r = api.route(logits, self.k_r, self.m_pad, self.seg_align) if self.routing is None else self._route_into(logits)
+        self.routing = r
+        api.fp8_quantize(x, dst_rows=r.dst_row, fanout=self.k_r, m_out=self.m_pad, codes=self.xc, s_out=self.xs)
+        api.w8a8_grouped_gemm(self.xc, self.xs, self.m_pad, self.c13, self.s13, 2 * I, H, E, r.offsets,
+                              seg_align=self.seg_align, epilogue=api.EPI_SWIGLU_BF16, row_token=r.row_token,
+                              row_gate=r.row_gate, out=self.h, amax_out=self.h_amax)
+        api.fp8_quantize(self.h, amax=self.h_amax, codes=self.hc, s_out=self.hs)
+        self.y.zero_()
+        api.w8a8_grouped_gemm(self.hc, self.hs, self.m_pad, self.c2, self.s2, H, I, E, r.offsets,
+                              seg_align=self.seg_align, epilogue=api.EPI_SCATTER_ADD_F32, row_token=r.row_token,
+                              row_gate=r.row_gate, out=self.y)
         return self.y
 
     _route_into = MoELayerW4A4._route_into

@@ -316,3 +316,44 @@ def test_moe_t16384_x_to_y_sampled(cuda):
     err = rel_fro(y[toks], want)
     print(f"moe_t16384_e128: sampled end-to-end relative Frobenius error {err:.2e}")
     assert err <= TOL
+
+
+def test_moe_layer_rac_half_of_channels(cuda):
+    """The pages' example of RAC on 50% of the channels (gist.science/it 2.2 B)
+    on the small MoE layer: k = 1024 of H = 2048 channels for X and 384 of
+    I = 768 for h, Y from X against the oracle's layer at the 2e-3 bar."""
+    from quantization_nvfp4_quantize_b200.moe import rac_channels
+    cfg = wl.CONFIGS["moe_t512_e8"]
+    x = wl.activations(cfg, 4)
+    logits = wl.router_logits(cfg, 4)
+    w13, w2 = wl.weights(cfg, 4)
+    kx, kh = rac_channels(50, cfg.hidden), rac_channels(50, cfg.inter)
+    assert (kx, kh) == (1024, 384)
+    layer = MoELayerW4A4(w13.to(cuda), w2.to(cuda), cfg.tokens, cfg.topk, kx, rac_k_h=kh)
+    y = layer.forward(x.to(cuda), logits.to(cuda)).cpu().numpy()
+    out = omoe.layer(_u16(x), logits.numpy(), omoe.quantize_weights(_u16(w13)), omoe.quantize_weights(_u16(w2)),
+                     cfg.topk, kx, kh)
+    check_selection(layer.xq.sel.cpu().numpy(), oracle.channel_score(out["xq"].resid), out["S_x"], kx)
+    err = rel_fro(y, out["Y"])
+    print(f"moe_t512_e8, RAC on 50% of channels: relative Frobenius error {err:.2e}")
+    assert err <= TOL
+
+
+def test_moe_layer_rac_second_pass(cuda):
+    """The small MoE layer with the second-pass NVFP4 RAC variant end to end
+    against the oracle's layer (rac_mode 'nvfp4') at the 2e-3 bar."""
+    cfg = wl.CONFIGS["moe_t512_e8"]
+    x = wl.activations(cfg, 8)
+    logits = wl.router_logits(cfg, 8)
+    w13, w2 = wl.weights(cfg, 8)
+    layer = MoELayerW4A4(w13.to(cuda), w2.to(cuda), cfg.tokens, cfg.topk, cfg.rac_k, rac_mode="nvfp4")
+    y = layer.forward(x.to(cuda), logits.to(cuda)).cpu().numpy()
+    out = omoe.layer(_u16(x), logits.numpy(), omoe.quantize_weights(_u16(w13)), omoe.quantize_weights(_u16(w2)),
+                     cfg.topk, cfg.rac_k, cfg.rac_k, rac_mode="nvfp4")
+    dst = layer.routing.dst_row.cpu().numpy()
+    rho = np_u16(layer.xq.r_sel)
+    for j in range(cfg.topk):
+        assert np.array_equal(rho[dst[:, j], :cfg.rac_k], out["rho_x"])
+    err = rel_fro(y, out["Y"])
+    print(f"moe_t512_e8, second-pass RAC: relative Frobenius error {err:.2e}")
+    assert err <= TOL

@@ -368,3 +368,56 @@ def test_near_boundary_sweep_matches_oracle(cuda):
                          want_score=True)
         torch.cuda.synchronize()
         assert np.array_equal(q.codes.cpu().numpy(), codes[g])
+
+
+@pytest.mark.parametrize("M,K,k", [(300, 2048, 1024), (129, 768, 768), (64, 4096, 2048)])
+def test_quantize_rac_percent_channels(cuda, M, K, k):
+    """RAC on "the top k% of channels" (50% and 100%): selection, scores and
+    residual operand bit-exact beyond the former 256-channel cap."""
+    rng = np.random.default_rng(M + K + k)
+    _quant_parity(cuda, gen_x(rng, M, K), k)
+
+
+def test_channel_major_gather_wide(cuda):
+    """The channel-major weight gather with more than 256 channels (chunked
+    over channels) equals the K-major gather and the oracle's e2m1 * sf."""
+    rng = np.random.default_rng(31)
+    E, N, K, k, ld = 2, 256, 1536, 700, 768
+    w = oracle.f32_to_bf16(rng.standard_normal((E, N, K)).astype(np.float32) * 0.02)
+    _, s_t, codes, scales = api.qdq_weights(to_bf16_dev(w, cuda), want_qdq=False, want_packed=True)
+    ccm, scm = api.weights_channel_major(codes, scales, N, K)
+    sel = np.sort(rng.choice(K, k, replace=False)).astype(np.int32)
+    seld = torch.from_numpy(sel).to(cuda)
+    a = np_u16(api.gather_weight_channels(codes, scales, N, K, seld, k, ld))
+    b = np_u16(api.gather_weight_channels_cm(ccm, scm, N, K, seld, k, ld))
+    assert np.array_equal(a, b)
+    assert np.all(b[:, :, k:] == 0)
+    for e in range(E):
+        ref = oracle.quantize(w[e])
+        q = np.empty((N, K), np.uint8)
+        q[:, 0::2] = ref.codes & 0xF
+        q[:, 1::2] = ref.codes >> 4
+        vals = oracle.e2m1_decode(q) * np.repeat(oracle.e4m3_decode(ref.sf), 16, axis=1)
+        assert np.array_equal(b[e, :, :k], oracle.f32_to_bf16(vals[:, sel].astype(np.float32)))
+
+
+@pytest.mark.parametrize("M,K,k,ld", [(300, 768, 32, 64), (129, 2048, 100, 128), (64, 4096, 2048, 2048)])
+def test_rac_second_pass_nvfp4_parity(cuda, M, K, k, ld):
+    """The second-pass RAC variant: the selected residual channels quantized
+    again to NVFP4 (own tensor scale, 16-channel blocks, last block padded);
+    the operand bit-exact against the oracle, padding columns zero."""
+    rng = np.random.default_rng(M + K + k)
+    x = gen_x(rng, M, K)
+    xd = to_bf16_dev(x, cuda)
+    q = api.quantize(xd, rac_k=k, rac_ld=ld, want_score=True)
+    s_r = torch.empty(1, dtype=torch.float32, device=cuda)
+    api.rac_residual_nvfp4(xd, q, k, ld, s_r_out=s_r)
+    torch.cuda.synchronize()
+    ref = oracle.quantize(x)
+    sel = q.sel.cpu().numpy()[:k]
+    check_selection(sel, oracle.channel_score(ref.resid), oracle.select_topk(oracle.channel_score(ref.resid), k), k)
+    rho2, s_r_ref = oracle.rac_residual_nvfp4(ref.resid, ref.s_t, sel)
+    assert s_r.item() == np.float32(s_r_ref)
+    got = np_u16(q.r_sel)
+    assert np.array_equal(got[:, :k], rho2)
+    assert np.all(got[:, k:] == 0)
