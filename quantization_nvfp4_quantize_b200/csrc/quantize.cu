@@ -135,8 +135,6 @@ __device__ __forceinline__ bool qwait(uint32_t bar, uint32_t parity, volatile in
     }
 }
 
-constexpr int QFAN_SLOTS = 4;         // per-warp ring of staged code rows for the fan-out bulk stores
-
 // Byte offset of scale entry (r, c) in the scale-factor layout, 32-bit
 // (callers keep rows x K/16 below 2^31).
 __device__ __forceinline__ uint32_t sf_off32(uint32_t r, uint32_t c, uint32_t K)
@@ -151,11 +149,13 @@ __device__ __forceinline__ uint32_t sf_off32(uint32_t r, uint32_t c, uint32_t K)
 // (a lane pair is one 16-element block).
 //   SCORE  accumulate the channels' residual sums of squares
 //   QDQ    write bf16(xhat) (weight fake quantization)
-// With dst_rows, the codes of a row (128 contiguous bytes per warp) are staged
-// in shared memory and written to each destination row by one bulk copy per
-// destination; the scale words go out as 4-byte stores, one per lane.
+//   FAN    write the codes and scales to the routed rows dst_rows instead
+// With dst_rows, each destination row gets the warp's codes as one coalesced
+// 128-byte line (a 4-byte store per lane) and its 4 scale words as 4-byte
+// stores, one per lane; the destinations' row offsets are looked up once per
+// tile.
 // Offsets inside a tensor are 32-bit (the host checks the sizes).
-template <bool SCORE, bool QDQ>
+template <bool SCORE, bool QDQ, bool FAN>
 __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __grid_constant__ CUtensorMap tm_x,
                                                                      QuantParams p)
 {
@@ -163,8 +163,8 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
     __shared__ uint64_t full_bar[QSTAGES], empty_bar[QSTAGES];
     __shared__ int abort_sm;
     __shared__ float4 btab[128];                                  // per E4M3 code: d, rlo, rhi, sf_h2
-    __shared__ int32_t fdst[QWORKERS][QRPW][32];                  // fan-out rows of a warp's 4 rows
-    __shared__ __align__(128) uint32_t fstage[QWORKERS][QFAN_SLOTS][32];   // staged code rows
+    __shared__ int32_t fdst[QWORKERS][QRPW][32];                  // fan-out rows of a warp's 4 rows (-1: none)
+    __shared__ uint32_t fsrow[QWORKERS][QRPW][32];                // their row parts of the scale-atom offset
     volatile int *abort_flag = &abort_sm;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
     uint8_t *codes = p.codes ? p.codes + g * p.codes_gstride : nullptr;
     uint8_t *scales = p.scales ? p.scales + g * p.scales_gstride : nullptr;
     __nv_bfloat16 *qdq = QDQ ? p.qdq + g * p.qdq_gstride : nullptr;
-    const int fanout = p.dst_rows ? p.fanout : 0;
+    const int fanout = FAN ? p.fanout : 0;
     const uint32_t M_out = (uint32_t)p.M_out;
 
     // E4M3 code -> the block's constants: a block scale takes at most 127
@@ -243,9 +243,10 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
     } else {
         // -------------------------------------------------------- workers
         const uint32_t kb0 = c >> 4;            // first block of the lane octet's 4-block group (lanes 8j)
-        const uint32_t code_bytes = min(QCHUNK, (int)(K - c0)) / 2;    // one row's codes in this chunk
         const uint32_t wcol = (c0 >> 4) + 4 * (lane & 3);          // fan-out: first scale column of word lane % 4
-        int fan_slot = 0;
+        const bool wcol_ok = wcol < (K >> 4);
+        const uint32_t wcol_off = sf_off32(0u, wcol, K);             // column part of the word's offset
+        const uint32_t code_col = c >> 1;
         for (int it = 0; it < n_iter; ++it) {
             const int st = it % QSTAGES;
             const uint32_t ph = (uint32_t)(it / QSTAGES) & 1u;
@@ -254,11 +255,16 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
             if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
             const uint8_t *tile = qsm + st * QTILE + warp * QPITCH + lane * 16;
             const uint32_t rt = r0 + (uint32_t)it * QROWS + (uint32_t)warp;   // this warp's first row of the tile
-            if (fanout) {
+            if (FAN) {
 #pragma unroll
                 for (int i = 0; i < QRPW; ++i) {
                     const uint32_t r = rt + (uint32_t)(i * QWORKERS);
-                    if (lane < fanout) fdst[warp][i][lane] = r < r1 ? p.dst_rows[(int64_t)r * fanout + lane] : -1;
+                    if (lane < fanout) {
+                        int32_t dst = r < r1 ? p.dst_rows[(int64_t)r * fanout + lane] : -1;
+                        if (dst >= 0 && (uint32_t)dst >= M_out) dst = -1;
+                        fdst[warp][i][lane] = dst;
+                        fsrow[warp][i][lane] = dst >= 0 ? sf_off32((uint32_t)dst, 0u, K) : 0u;
+                    }
                 }
                 __syncwarp();
             }
@@ -299,33 +305,24 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
                 // the 4 scale codes of blocks kb0..kb0+3 on lanes 8j
                 uint32_t sw = sf_code | (__shfl_down_sync(0xffffffffu, sf_code, 2) << 8);
                 sw |= __shfl_down_sync(0xffffffffu, sw, 4) << 16;
-                if (!fanout) {
+                if (!FAN) {
                     if (active) {
                         *reinterpret_cast<uint32_t *>(codes + r * (K >> 1) + (c >> 1)) = cw;
                         if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(scales + sf_off32(r, kb0, K)) = sw;
                     }
-                    continue;
-                }
-                // fan-out: stage the row's codes, one bulk copy per destination
-                uint32_t *slot = fstage[warp][fan_slot];
-                if (lane < fanout) ptx::bulk_wait_read<QFAN_SLOTS - 1>();
-                __syncwarp();
-                slot[lane] = cw;
-                ptx::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane < fanout) {
-                    const int32_t dst = fdst[warp][i][lane];
-                    if (dst >= 0 && (uint32_t)dst < M_out)
-                        ptx::bulk_store(codes + (uint64_t)dst * (K >> 1) + (c0 >> 1), ptx::smem_u32(slot), code_bytes);
-                    ptx::bulk_commit();
-                }
-                fan_slot = (fan_slot + 1) % QFAN_SLOTS;
-                // scale words: lane l writes word l % 4 of destination l / 4 (+ 8 per round)
-                const uint32_t word = __shfl_sync(0xffffffffu, sw, (lane & 3) * 8);
-                for (int d = lane >> 2; d < fanout; d += 8) {
-                    const int32_t dst = fdst[warp][i][d];
-                    if (dst >= 0 && (uint32_t)dst < M_out && wcol < (K >> 4))
-                        *reinterpret_cast<uint32_t *>(scales + sf_off32((uint32_t)dst, wcol, K)) = word;
+                } else {
+                    // fan-out: the row's codes, one 128-byte line per destination
+                    for (int d = 0; d < fanout; ++d) {
+                        const int32_t dst = fdst[warp][i][d];
+                        if (dst >= 0 && active)
+                            *reinterpret_cast<uint32_t *>(codes + (uint64_t)(uint32_t)dst * (K >> 1) + code_col) = cw;
+                    }
+                    // scale words: lane l writes word l % 4 of destination l / 4 (+ 8 per round)
+                    const uint32_t word = __shfl_sync(0xffffffffu, sw, (lane & 3) * 8);
+                    for (int d = lane >> 2; d < fanout; d += 8) {
+                        if (fdst[warp][i][d] >= 0 && wcol_ok)
+                            *reinterpret_cast<uint32_t *>(scales + fsrow[warp][i][d] + wcol_off) = word;
+                    }
                 }
             }
             if (SCORE) {
@@ -340,7 +337,6 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty_bar[st]));
         }
-        if (fanout && lane < fanout) ptx::bulk_wait_all();        // staged rows read and written
     }
 
     if (SCORE) {
@@ -767,7 +763,7 @@ static int64_t row_groups(int64_t M, int64_t rpc) { return std::max<int64_t>(1, 
 // Builds the TMA map over x ([rows_total x K] bf16, row stride ldx) and
 // launches k_quantize.  `fallback` is any valid 16-byte aligned device
 // address, used as the map's base when x has no rows (no copy is issued then).
-template <bool SCORE, bool QDQ>
+template <bool SCORE, bool QDQ, bool FAN>
 static nvfp4_status launch_quantize_t(const CUtensorMap &tm, const QuantParams &p, dim3 grid, size_t smem,
                                       cudaStream_t st)
 {
@@ -776,12 +772,12 @@ static nvfp4_status launch_quantize_t(const CUtensorMap &tm, const QuantParams &
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return check_launch("k_quantize: device");
     std::call_once(once[dev], [&] {
-        attr_err[dev] = cudaFuncSetAttribute(k_quantize<SCORE, QDQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err[dev] = cudaFuncSetAttribute(k_quantize<SCORE, QDQ, FAN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)QSMEM);
     });
     if (attr_err[dev] != cudaSuccess) return set_error(NVFP4_ERR_CUDA, "k_quantize: smem attribute: %s",
                                                        cudaGetErrorString(attr_err[dev]));
-    k_quantize<SCORE, QDQ><<<grid, QTHREADS, smem, st>>>(tm, p);
+    k_quantize<SCORE, QDQ, FAN><<<grid, QTHREADS, smem, st>>>(tm, p);
     return check_launch("k_quantize");
 }
 
@@ -800,9 +796,15 @@ static nvfp4_status launch_quantize(bool score, const void *x, int64_t rows_tota
                       CU_TENSOR_MAP_SWIZZLE_NONE))
         return set_error(NVFP4_ERR_CUDA, "k_quantize: tensor map encoding failed");
     const size_t smem = QSMEM;
-    if (p.qdq) return launch_quantize_t<false, true>(tm, p, grid, smem, st);
-    if (score) return launch_quantize_t<true, false>(tm, p, grid, smem, st);
-    return launch_quantize_t<false, false>(tm, p, grid, smem, st);
+    const bool fan = p.dst_rows != nullptr;
+    if (p.qdq) {
+        NVFP4_REQUIRE(!fan, NVFP4_ERR_INVALID_ARG, "k_quantize: the QDQ output has no routed-row form");
+        return launch_quantize_t<false, true, false>(tm, p, grid, smem, st);
+    }
+    if (score) return fan ? launch_quantize_t<true, false, true>(tm, p, grid, smem, st)
+                          : launch_quantize_t<true, false, false>(tm, p, grid, smem, st);
+    return fan ? launch_quantize_t<false, false, true>(tm, p, grid, smem, st)
+               : launch_quantize_t<false, false, false>(tm, p, grid, smem, st);
 }
 
 }  // namespace nvfp4
