@@ -100,6 +100,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the trainer-side W4A16 line of the default run")
     ap.add_argument("--no-formats", action="store_true", help="skip the W4A4 / W8A8 / BF16 grouped-GEMM table")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the layer-error sweep over RAC channels and outliers")
     return ap.parse_args()
 
 
@@ -343,11 +344,37 @@ def run_ours(args):
         torch.cuda.empty_cache()
         out["gemm_formats"] = run_formats(args, dev)
         out["gpu_launches"] += out["gemm_formats"].pop("_launches")
+    if not args.no_sweep:
+        # accuracy side of RAC: the error it leaves on one dense layer, by
+        # compensated channel share and outlier strength (untimed)
+        torch.cuda.empty_cache()
+        out["error_sweep"] = run_error_sweep(args, dev)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg, seed=args.seed, n_experts=64)
     if rank == 0:
         print(json.dumps(out), flush=True)
     return out
+
+
+def run_error_sweep(args, dev):
+    """err(k) = ||Y_RAC(k) - X What^T||_F / ||X What^T||_F of one dense layer
+    for RAC on k% of the input channels (bf16 residual and the NVFP4 second
+    pass) and outlier channels of growing strength."""
+    from quantization_nvfp4_quantize_b200 import workloads as wl
+    from quantization_nvfp4_quantize_b200.sweep import LayerErrorProbe, rac_channels
+    sw = wl.SWEEP
+    T, K, N = sw["tokens"], sw["channels"], sw["out"]
+    ks = [rac_channels(p_, K) for p_ in sw["percents"]]
+    probe = LayerErrorProbe(wl.dense_weight(N, K, args.seed, device=dev), T)
+    res = {"metric": "||Y_RAC(k) - X What^T||_F / ||X What^T||_F",
+           "workload": f"dense T={T} K={K} N={N}; X N(0,1) with {int(round(sw['outlier_frac'] * K))} channels "
+                       "x alpha; W N(0,0.02) in NVFP4",
+           "percents": list(sw["percents"]), "k": ks, "bf16_residual": {}, "nvfp4_second_pass": {}}
+    for a in sw["alphas"]:
+        x = wl.outlier_activations(T, K, a, args.seed, frac=sw["outlier_frac"], device=dev)
+        res["bf16_residual"][f"alpha_{a:g}"] = [float(f"{e:.4g}") for e in probe.errors(x, ks, "bf16")]
+        res["nvfp4_second_pass"][f"alpha_{a:g}"] = [float(f"{e:.4g}") for e in probe.errors(x, ks, "nvfp4")]
+    return res
 
 
 def run_formats(args, dev):

@@ -121,6 +121,33 @@ def weights(cfg: LayerConfig, seed: int, device="cpu"):
     return w13, w2
 
 
+# Layer-error sweep (one dense layer): outlier strength alpha scales a fixed
+# 1% of the input channels; RAC channel counts as percentages of K.
+SWEEP = {"tokens": 4096, "channels": 4096, "out": 4096, "outlier_frac": 0.01,
+         "alphas": (1.0, 5.0, 20.0, 50.0), "percents": (0, 1, 2, 5, 10, 25, 50, 100)}
+
+
+def outlier_activations(tokens: int, channels: int, alpha: float, seed: int, frac: float = 0.01,
+                        device="cpu") -> torch.Tensor:
+    """X bf16 [tokens x channels]: N(0,1) with round(frac * channels) seeded
+    channels multiplied by ``alpha`` (alpha = 1: no outliers).  The same
+    channels for every alpha of a seed."""
+    g = _gen(seed, 11, device)
+    x = torch.randn(tokens, channels, generator=g, device=device, dtype=torch.float32)
+    n = int(round(frac * channels))
+    if n and alpha != 1.0:
+        gc = _gen(seed, 12, "cpu")
+        ch = torch.randperm(channels, generator=gc)[:n]
+        x[:, ch.to(device)] *= float(alpha)
+    return x.to(torch.bfloat16)
+
+
+def dense_weight(n_out: int, n_in: int, seed: int, device="cpu") -> torch.Tensor:
+    """W bf16 [n_out x n_in] (K-major rows), N(0, 0.02)."""
+    g = _gen(seed, 13, device)
+    return (torch.randn(n_out, n_in, generator=g, device=device) * 0.02).to(torch.bfloat16)
+
+
 def padded_rows_bound(cfg: LayerConfig) -> int:
     """Upper bound on the expert-grouped routed rows once every expert's
     segment is padded to a multiple of 128: T*k_r + E*127, rounded up to 128."""
