@@ -146,6 +146,35 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, i
                             void *stream);
 
 /* --------------------------------------------------------------------------
+ * nvfp4_quantize_experts -- nvfp4_quantize with one RAC channel set per
+ * expert (READING: the pages select one binary mask of the top-k channels by
+ * residual magnitude per GEMM input, gist.science/it 2.2 B; here each
+ * expert's GEMM input gets the mask of its own rows).  x holds routed rows
+ * in the expert-grouped layout of moe_route (expert e owns rows
+ * [offsets[e], offsets[e+1]), segments padded to seg_align with zero rows;
+ * rows >= offsets[E] are ignored), e.g. h from the gate/up GEMM or X from
+ * moe_routed_rows_bf16.
+ *   one tensor scale s_t over all rows (s_t_in / amax_in / amax pass as for
+ *   nvfp4_quantize); codes and scales for every row (M_out = M, no fan-out);
+ *   score_dev   optional float64 [E x K]: score[e,c] = sum over e's rows of
+ *               R[r,c]^2 (NULL: kept in the workspace);
+ *   sel_dev     int32 [E x rac_k]: expert e's channels, ascending;
+ *   r_sel_dev   bf16 [M x rac_ld]: rho[r, j] = bf16(R[r, S_e(r)[j]] / s_t),
+ *               zero for j >= rac_k.
+ * 1 <= E <= 256, seg_align 128 or 256, M % seg_align == 0, 1 <= rac_k <= K,
+ * rac_ld % 64 == 0; K, ldx and alignment as for nvfp4_quantize.
+ * workspace: nvfp4_quantize_experts_workspace_size(M, K, E, seg_align).
+ * -------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_quantize_experts_workspace_size(int64_t M, int64_t K, int32_t E, int32_t seg_align);
+
+NVFP4_API nvfp4_status nvfp4_quantize_experts(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
+                                    const int32_t *offsets_dev, int32_t E, int32_t seg_align,
+                                    const float *s_t_in_dev, const float *amax_in_dev, float *s_t_out_dev,
+                                    uint8_t *codes_dev, uint8_t *scales_dev, double *score_dev,
+                                    int32_t rac_k, int32_t rac_ld, int32_t *sel_dev, void *r_sel_dev,
+                                    int32_t *dev_status, void *workspace, size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
  * nvfp4_quantize_noalloc -- nvfp4_quantize without a caller workspace.  The
  * QUADS pages have no counterpart to this entry point; it exists for callers
  * that cannot allocate device memory at the moment they quantize: a plug-in
@@ -297,6 +326,14 @@ NVFP4_API nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_d
                                                        int32_t E, int64_t N, int64_t K, const int32_t *sel_dev,
                                                        int32_t k, int32_t ld, void *w_sel_dev, void *stream);
 
+/* nvfp4_gather_weight_channels_cm_experts -- the same with one channel set
+ * per expert (per-expert RAC, see nvfp4_quantize_experts): sel_dev is int32
+ * [E x k] and expert e gathers the channels sel[e*k .. e*k + k). */
+NVFP4_API nvfp4_status nvfp4_gather_weight_channels_cm_experts(const uint8_t *codes_cm_dev,
+                                                               const uint8_t *scales_cm_dev, int32_t E, int64_t N,
+                                                               int64_t K, const int32_t *sel_dev, int32_t k,
+                                                               int32_t ld, void *w_sel_dev, void *stream);
+
 /* --------------------------------------------------------------------------
  * moe_w4a4_grouped_gemm_rac -- the native W4A4 block-scaled grouped expert
  * GEMM with Residual Activation Compensation folded into the same
@@ -396,6 +433,16 @@ NVFP4_API nvfp4_status moe_bf16_grouped_gemm(
 NVFP4_API nvfp4_status moe_gather_rows_bf16(const void *x_dev, int64_t T, int64_t K, int64_t ldx,
                                             const int32_t *dst_rows_dev, int32_t fanout, void *out_dev,
                                             int64_t ld_out, int64_t M_out, void *stream);
+
+/* moe_routed_rows_bf16 -- the complete routed copy of x: every row r < M_out
+ * of out (bf16 [M_out x ld_out]) receives token row row_token[r] of x (bf16
+ * [T x ldx]), or zeros where row_token[r] < 0 (segment padding), so rows a
+ * previous routing left behind never survive.  Used by per-expert RAC on the
+ * gate/up input.  K % 8 == 0, ldx and ld_out >= K and multiples of 8,
+ * pointers 16-byte aligned, M_out < 2^31. */
+NVFP4_API nvfp4_status moe_routed_rows_bf16(const void *x_dev, int64_t T, int64_t K, int64_t ldx,
+                                            const int32_t *row_token_dev, void *out_dev, int64_t ld_out,
+                                            int64_t M_out, void *stream);
 
 /* --------------------------------------------------------------------------
  * fp8_quantize / moe_w8a8_grouped_gemm -- the FP8 comparison path: the pages

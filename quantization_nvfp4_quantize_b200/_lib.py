@@ -61,6 +61,14 @@ SIGNATURES = {
     "moe_w8a8_grouped_gemm": (c_int32, [c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_int64, c_int64, c_int32,
                                         c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_void_p,
                                         c_void_p, c_void_p]),
+    "nvfp4_quantize_experts_workspace_size": (c_size_t, [c_int64, c_int64, c_int32, c_int32]),
+    "nvfp4_quantize_experts": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int32, c_int32, c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "nvfp4_gather_weight_channels_cm_experts": (c_int32, [c_void_p, c_void_p, c_int32, c_int64, c_int64, c_void_p,
+                                                          c_int32, c_int32, c_void_p, c_void_p]),
+    "moe_routed_rows_bf16": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_int64, c_int64,
+                                       c_void_p]),
     "nvfp4_debug_gemm_wait_expiry": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
                                                c_int64, c_int64, c_int32, c_void_p, c_int32, c_void_p, c_void_p,
                                                c_void_p, c_int64, c_void_p, c_int64, c_void_p]),

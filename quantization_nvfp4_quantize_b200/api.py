@@ -87,6 +87,36 @@ def quantize(x: torch.Tensor, *, rac_k: int = 0, rac_ld: int | None = None, s_t:
     return out
 
 
+def quantize_experts(x: torch.Tensor, offsets: torch.Tensor, E: int, seg_align: int, *, rac_k: int,
+                     rac_ld: int | None = None, s_t: torch.Tensor | None = None, amax: torch.Tensor | None = None,
+                     want_score: bool = False, out: Quantized | None = None, workspace: torch.Tensor | None = None,
+                     dev_status: torch.Tensor | None = None) -> Quantized:
+    """nvfp4_quantize_experts on expert-grouped routed rows bf16 [M, K]: one
+    RAC channel set per expert (sel [E, rac_k], score [E, K])."""
+    lib = _lib.load()
+    assert x.dtype == BF16 and x.dim() == 2 and x.stride(1) == 1
+    M, K = x.shape
+    dev = x.device
+    if rac_ld is None:
+        rac_ld = -(-rac_k // 64) * 64
+    if out is None:
+        out = Quantized(
+            codes=torch.empty(M, K // 2, dtype=U8, device=dev),
+            scales=torch.empty(scale_bytes(M, K), dtype=U8, device=dev),
+            s_t=torch.empty(1, dtype=F32, device=dev),
+            score=torch.empty(E, K, dtype=F64, device=dev) if want_score else None,
+            sel=torch.empty(E, rac_k, dtype=I32, device=dev),
+            r_sel=torch.empty(M, rac_ld, dtype=BF16, device=dev),
+        )
+    if workspace is None:
+        workspace = _ws(lib.nvfp4_quantize_experts_workspace_size(M, K, E, seg_align), dev)
+    check(lib.nvfp4_quantize_experts(_p(x), M, K, x.stride(0), _p(offsets), E, seg_align, _p(s_t), _p(amax),
+                                     _p(out.s_t), _p(out.codes), _p(out.scales), _p(out.score), rac_k, rac_ld,
+                                     _p(out.sel), _p(out.r_sel), _p(dev_status), _p(workspace), workspace.numel(),
+                                     _stream(dev)))
+    return out
+
+
 def qdq_weights(w: torch.Tensor, *, want_qdq: bool = True, want_packed: bool = False):
     """nvfp4_qdq_weights on bf16 [G, rows, cols] (or [rows, cols]).
     Returns (w_qdq or None, s_t [G], codes or None, scales or None)."""
@@ -173,6 +203,19 @@ def gather_weight_channels_cm(codes_cm: torch.Tensor, scales_cm: torch.Tensor, N
     return out
 
 
+def gather_weight_channels_cm_experts(codes_cm: torch.Tensor, scales_cm: torch.Tensor, N: int, K: int,
+                                      sel: torch.Tensor, k: int, ld: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """nvfp4_gather_weight_channels_cm_experts: expert e gathers sel[e, :k]."""
+    lib = _lib.load()
+    E = codes_cm.shape[0]
+    assert sel.dtype == I32 and sel.numel() >= E * k
+    if out is None:
+        out = torch.empty(E, N, ld, dtype=BF16, device=codes_cm.device)
+    check(lib.nvfp4_gather_weight_channels_cm_experts(_p(codes_cm), _p(scales_cm), E, N, K, _p(sel), k, ld, _p(out),
+                                                      _stream(codes_cm.device)))
+    return out
+
+
 def grouped_gemm(a_codes, a_scales, a_s_t, m_pad_max, b_codes, b_scales, b_s_t, N, K, E, offsets, *,
                  seg_align=128, rac_ld=0, rho=None, w_sel=None, epilogue=EPI_STORE_F32, row_token=None, row_gate=None,
                  out=None, ld_out=None, amax_out=None, dev_status=None):
@@ -211,6 +254,18 @@ def gather_rows_bf16(x: torch.Tensor, dst_rows: torch.Tensor, m_out: int, *, out
         out = torch.zeros(m_out, K, dtype=BF16, device=x.device)
     check(lib.moe_gather_rows_bf16(_p(x), T, K, x.stride(0), _p(dst_rows), dst_rows.shape[1], _p(out), out.stride(0),
                                    m_out, _stream(x.device)))
+    return out
+
+
+def routed_rows_bf16(x: torch.Tensor, row_token: torch.Tensor, m_out: int, *, out=None):
+    """moe_routed_rows_bf16: out[r] = x[row_token[r]], zero rows for padding."""
+    lib = _lib.load()
+    assert x.dtype == BF16 and x.dim() == 2 and x.stride(1) == 1
+    T, K = x.shape
+    if out is None:
+        out = torch.empty(m_out, K, dtype=BF16, device=x.device)
+    check(lib.moe_routed_rows_bf16(_p(x), T, K, x.stride(0), _p(row_token), _p(out), out.stride(0), m_out,
+                                   _stream(x.device)))
     return out
 
 

@@ -370,6 +370,21 @@ __global__ void k_score_reduce(const double *__restrict__ partials, int64_t P, i
     score[c] = s;
 }
 
+// Per-expert scores from row-group partials: row group q covers rows
+// [q*rpc, (q+1)*rpc), inside one expert segment (segments are multiples of
+// rpc); score[e, c] sums expert e's groups in order.
+__global__ void k_score_reduce_experts(const double *__restrict__ partials, const int32_t *__restrict__ offsets,
+                                      int64_t rpc, int64_t K, double *__restrict__ score)
+{
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int e = blockIdx.y;
+    if (c >= K) return;
+    const int64_t q0 = offsets[e] / rpc, q1 = offsets[e + 1] / rpc;
+    double s = 0.0;
+    for (int64_t q = q0; q < q1; ++q) s += partials[q * K + c];
+    score[(int64_t)e * K + c] = s;
+}
+
 // ---------------------------------------------------------------- top-k
 
 __device__ __forceinline__ int block_exclusive_scan(int v, int *smem_warp, int &total)
@@ -414,6 +429,8 @@ __global__ void __launch_bounds__(1024) k_select_topk(const double *__restrict__
     __shared__ int s_digit, s_rem;
     const int tid = threadIdx.x;
     if (k <= 0) return;
+    score += (int64_t)blockIdx.x * K;                 // one score vector (and set) per block
+    sel += (int64_t)blockIdx.x * k;
     for (int i = tid; i < K; i += blockDim.x) keys[i] = (unsigned long long)__double_as_longlong(score[i]);
     if (tid == 0) s_rem = k;
     __syncthreads();
@@ -497,13 +514,23 @@ __global__ void __launch_bounds__(256) k_rac_residual(
     const __nv_bfloat16 *__restrict__ x, int64_t ldx, int64_t M, int64_t K,
     const int32_t *__restrict__ m_valid, const float *__restrict__ s_t_ptr,
     const int32_t *__restrict__ sel, int k, int ld,
-    const int32_t *__restrict__ dst_rows, int fanout, int64_t M_out, __nv_bfloat16 *__restrict__ r_sel)
+    const int32_t *__restrict__ dst_rows, int fanout, int64_t M_out, __nv_bfloat16 *__restrict__ r_sel,
+    const int32_t *__restrict__ expert_offsets, int E)
 {
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     int64_t Me = M;
     if (m_valid) Me = min(Me, (int64_t)max(*m_valid, 0));
     if (r >= Me) return;
+    if (expert_offsets) {
+        // per-expert sets: row r belongs to expert e, offsets[e] <= r < offsets[e+1]
+        int lo = 0, hi = E;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (expert_offsets[mid] <= r) lo = mid; else hi = mid;
+        }
+        sel += (int64_t)lo * k;
+    }
     const float s_t = *s_t_ptr;
     const float2 r6 = recip_bracket(__fmul_rn(6.0f, s_t));
     const int nd = dst_rows ? fanout : 1;
@@ -679,7 +706,7 @@ constexpr int GCM_J = 256;                           // output channels per CTA 
 __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__restrict__ codes_cm,
                                                               const uint8_t *__restrict__ scales_cm, int64_t N,
                                                               int64_t K, const int32_t *__restrict__ sel, int k,
-                                                              int ld, __nv_bfloat16 *__restrict__ out)
+                                                              int ld, __nv_bfloat16 *__restrict__ out, int sel_stride)
 {
     extern __shared__ float gtile[];                   // [GCM_N features][cw channels of this chunk]
     __shared__ float e4[128];                          // E4M3 code -> value (weight scales are non-negative)
@@ -691,7 +718,7 @@ __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__r
     const int j0 = blockIdx.z * GCM_J;
     const int cw = min(GCM_J, ld - j0);
     const int kc = max(0, min(k - j0, cw));
-    sel += j0;
+    sel += e * sel_stride + j0;                          // sel_stride 0: one set for every expert
     if (threadIdx.x < 128) e4[threadIdx.x] = e4m3_to_f32(threadIdx.x);
     for (int j = threadIdx.x; j < kc; j += blockDim.x) ssel[j] = sel[j];
     __syncthreads();
@@ -918,9 +945,110 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
             unsigned blocks = (unsigned)((M + 7) / 8);
             k_rac_residual<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, s_t_used,
                                                    sel_dev, rac_k, rac_ld, dst_rows_dev,
-                                                   dst_rows_dev ? fanout : 1, M_out, (__nv_bfloat16 *)r_sel_dev);
+                                                   dst_rows_dev ? fanout : 1, M_out, (__nv_bfloat16 *)r_sel_dev,
+                                                   nullptr, 0);
             if (check_launch("k_rac_residual") != NVFP4_OK) return NVFP4_ERR_CUDA;
         }
+    }
+    return NVFP4_OK;
+}
+
+extern "C" size_t nvfp4_quantize_experts_workspace_size(int64_t M, int64_t K, int32_t E, int32_t seg_align)
+{
+    if (M < 0 || K <= 0 || E < 1 || (seg_align != 128 && seg_align != 256)) return 0;
+    const int64_t P = std::max<int64_t>(1, (M + seg_align - 1) / seg_align);
+    return 256 + (size_t)(P * K + (int64_t)E * K) * sizeof(double);
+}
+
+extern "C" nvfp4_status nvfp4_quantize_experts(const void *x_dev, int64_t M, int64_t K, int64_t ldx,
+                                               const int32_t *offsets_dev, int32_t E, int32_t seg_align,
+                                               const float *s_t_in_dev, const float *amax_in_dev,
+                                               float *s_t_out_dev, uint8_t *codes_dev, uint8_t *scales_dev,
+                                               double *score_dev, int32_t rac_k, int32_t rac_ld,
+                                               int32_t *sel_dev, void *r_sel_dev, int32_t *dev_status,
+                                               void *workspace, size_t workspace_bytes, void *stream)
+{
+    cudaStream_t st = (cudaStream_t)stream;
+    NVFP4_REQUIRE(M >= 0 && K > 0, NVFP4_ERR_INVALID_ARG, "nvfp4_quantize_experts: bad sizes");
+    NVFP4_REQUIRE(E >= 1 && E <= 256 && offsets_dev, NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_quantize_experts: need 1 <= E <= 256 and the expert offsets");
+    NVFP4_REQUIRE(seg_align == 128 || seg_align == 256, NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_quantize_experts: seg_align must be 128 or 256");
+    NVFP4_REQUIRE(M % seg_align == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_quantize_experts: M must be a multiple of seg_align");
+    NVFP4_REQUIRE(s_t_out_dev && (M == 0 || (x_dev && codes_dev && scales_dev)), NVFP4_ERR_INVALID_ARG,
+                  "nvfp4_quantize_experts: x, s_t_out, codes and scales are required");
+    NVFP4_REQUIRE(K % 64 == 0 && K <= 16384, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_quantize_experts: K must be a multiple of 64 and <= 16384");
+    NVFP4_REQUIRE(ldx >= K && ldx % 8 == 0, NVFP4_ERR_ALIGNMENT,
+                  "nvfp4_quantize_experts: ldx must be >= K and a multiple of 8");
+    NVFP4_REQUIRE(aligned16(x_dev) && aligned16(codes_dev) && aligned16(scales_dev), NVFP4_ERR_ALIGNMENT,
+                  "nvfp4_quantize_experts: x, codes and scales must be 16-byte aligned");
+    NVFP4_REQUIRE(rac_k >= 1 && rac_k <= K && sel_dev && r_sel_dev && rac_ld >= rac_k && rac_ld % 64 == 0,
+                  NVFP4_ERR_UNSUPPORTED_SHAPE,
+                  "nvfp4_quantize_experts: need 1 <= rac_k <= K, sel, r_sel, rac_ld >= rac_k, rac_ld % 64 == 0");
+    NVFP4_REQUIRE(aligned16(r_sel_dev), NVFP4_ERR_ALIGNMENT, "nvfp4_quantize_experts: r_sel must be 16-byte aligned");
+    const size_t need = nvfp4_quantize_experts_workspace_size(M, K, E, seg_align);
+    NVFP4_REQUIRE(workspace && workspace_bytes >= need && aligned16(workspace), NVFP4_ERR_WORKSPACE,
+                  "nvfp4_quantize_experts: workspace of %zu bytes (16-byte aligned) required", need);
+    const int32_t *m_valid_dev = offsets_dev + E;               // rows past the last segment are not routed
+    const unsigned int *amax_bits = amax_in_dev ? reinterpret_cast<const unsigned int *>(amax_in_dev)
+                                                : reinterpret_cast<unsigned int *>(workspace);
+    const int64_t nch = (K + QCHUNK - 1) / QCHUNK;
+    const int64_t P = std::max<int64_t>(1, M / seg_align);
+    double *partials = reinterpret_cast<double *>(reinterpret_cast<char *>(workspace) + 256);
+    double *score = score_dev ? score_dev : partials + P * K;
+    if (!s_t_in_dev && !amax_in_dev) {
+        unsigned int *slot = reinterpret_cast<unsigned int *>(workspace);
+        if (cudaMemsetAsync(slot, 0, 4, st) != cudaSuccess) return check_launch("nvfp4_quantize_experts: memset");
+        if (M > 0) {
+            int blocks = (int)std::min<int64_t>((int64_t)num_sms() * 8, std::max<int64_t>(1, (M * K / 8 + 255) / 256));
+            k_amax<<<dim3(blocks, 1), 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, 0, slot);
+            if (check_launch("k_amax") != NVFP4_OK) return NVFP4_ERR_CUDA;
+        }
+    }
+    // one row group per seg_align rows: every group lies in one expert's segment
+    QuantParams p{};
+    p.ldx = ldx; p.M = M; p.K = K;
+    p.m_valid = m_valid_dev;
+    p.s_t_in = s_t_in_dev;
+    p.amax_bits = amax_bits;
+    p.s_t_out = s_t_out_dev;
+    p.dst_rows = nullptr;
+    p.fanout = 1;
+    p.M_out = M;
+    p.codes = codes_dev;
+    p.scales = scales_dev;
+    p.qdq = nullptr;
+    p.partials = partials;
+    p.rows_per_cta = seg_align;
+    p.dev_status = dev_status;
+    if (launch_quantize(true, x_dev, M, workspace, p, dim3((unsigned)nch, (unsigned)P, 1), st) != NVFP4_OK)
+        return NVFP4_ERR_CUDA;
+    k_score_reduce_experts<<<dim3((unsigned)((K + 255) / 256), (unsigned)E), 256, 0, st>>>(partials, offsets_dev,
+                                                                                          seg_align, K, score);
+    if (check_launch("k_score_reduce_experts") != NVFP4_OK) return NVFP4_ERR_CUDA;
+    {
+        static std::once_flag once[64];
+        static cudaError_t attr_err[64];
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            return check_launch("nvfp4_quantize_experts: device");
+        std::call_once(once[dev], [&] {
+            attr_err[dev] = cudaFuncSetAttribute(k_select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, 16384 * 8);
+        });
+        if (attr_err[dev] != cudaSuccess)
+            return set_error(NVFP4_ERR_CUDA, "nvfp4_quantize_experts: smem attribute: %s",
+                             cudaGetErrorString(attr_err[dev]));
+    }
+    k_select_topk<<<(unsigned)E, 1024, (size_t)K * sizeof(unsigned long long), st>>>(score, (int)K, rac_k, sel_dev);
+    if (check_launch("k_select_topk") != NVFP4_OK) return NVFP4_ERR_CUDA;
+    if (M > 0) {
+        const float *s_t_used = s_t_in_dev ? s_t_in_dev : s_t_out_dev;
+        k_rac_residual<<<(unsigned)((M + 7) / 8), 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev,
+                                                               s_t_used, sel_dev, rac_k, rac_ld, nullptr, 1, M,
+                                                               (__nv_bfloat16 *)r_sel_dev, offsets_dev, E);
+        if (check_launch("k_rac_residual") != NVFP4_OK) return NVFP4_ERR_CUDA;
     }
     return NVFP4_OK;
 }
@@ -1051,9 +1179,9 @@ extern "C" nvfp4_status nvfp4_weights_channel_major(const uint8_t *codes_dev, co
     return check_launch("k_weights_channel_major");
 }
 
-extern "C" nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_dev, const uint8_t *scales_cm_dev,
-                                                        int32_t E, int64_t N, int64_t K, const int32_t *sel_dev,
-                                                        int32_t k, int32_t ld, void *w_sel_dev, void *stream)
+static nvfp4_status gather_cm(const uint8_t *codes_cm_dev, const uint8_t *scales_cm_dev, int32_t E, int64_t N,
+                              int64_t K, const int32_t *sel_dev, int32_t k, int32_t ld, void *w_sel_dev,
+                              int sel_stride, void *stream)
 {
     NVFP4_REQUIRE(codes_cm_dev && scales_cm_dev && w_sel_dev && (k == 0 || sel_dev), NVFP4_ERR_INVALID_ARG,
                   "nvfp4_gather_weight_channels_cm: null pointer");
@@ -1080,8 +1208,23 @@ extern "C" nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_
     }
     dim3 grid((unsigned)((N + GCM_N - 1) / GCM_N), (unsigned)E, (unsigned)((ld + GCM_J - 1) / GCM_J));
     k_gather_w_channels_cm<<<grid, 256, smem, (cudaStream_t)stream>>>(codes_cm_dev, scales_cm_dev, N, K, sel_dev, k,
-                                                                    ld, (__nv_bfloat16 *)w_sel_dev);
+                                                                    ld, (__nv_bfloat16 *)w_sel_dev, sel_stride);
     return check_launch("k_gather_w_channels_cm");
+}
+
+extern "C" nvfp4_status nvfp4_gather_weight_channels_cm(const uint8_t *codes_cm_dev, const uint8_t *scales_cm_dev,
+                                                        int32_t E, int64_t N, int64_t K, const int32_t *sel_dev,
+                                                        int32_t k, int32_t ld, void *w_sel_dev, void *stream)
+{
+    return gather_cm(codes_cm_dev, scales_cm_dev, E, N, K, sel_dev, k, ld, w_sel_dev, 0, stream);
+}
+
+extern "C" nvfp4_status nvfp4_gather_weight_channels_cm_experts(const uint8_t *codes_cm_dev,
+                                                                const uint8_t *scales_cm_dev, int32_t E, int64_t N,
+                                                                int64_t K, const int32_t *sel_dev, int32_t k,
+                                                                int32_t ld, void *w_sel_dev, void *stream)
+{
+    return gather_cm(codes_cm_dev, scales_cm_dev, E, N, K, sel_dev, k, ld, w_sel_dev, k, stream);
 }
 
 // ------------------------------------------------ FP8 E4M3 (comparison)

@@ -295,3 +295,37 @@ extern "C" nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E,
                                                   offsets_dev, dst_row_dev, row_token_dev, row_gate_dev);
     return check_launch("k_route_place");
 }
+
+// Every routed row r < M_out gets token row_token[r] of x, or zeros for a
+// padding row (row_token < 0): the copy is complete whatever the routing
+// left in the buffer before.
+__global__ void __launch_bounds__(256) k_routed_rows_bf16(const uint4 *__restrict__ x, int64_t T, int64_t K,
+                                                          int64_t ldx, const int32_t *__restrict__ row_token,
+                                                          uint4 *__restrict__ out, int64_t ld_out)
+{
+    const int64_t r = blockIdx.x;
+    const int64_t col = ((int64_t)blockIdx.y * 256 + threadIdx.x) * 8;
+    if (col >= K) return;
+    const int32_t t = row_token[r];
+    const uint4 v = (t >= 0 && t < T) ? x[((int64_t)t * ldx + col) >> 3] : make_uint4(0u, 0u, 0u, 0u);
+    out[(r * ld_out + col) >> 3] = v;
+}
+
+extern "C" nvfp4_status moe_routed_rows_bf16(const void *x_dev, int64_t T, int64_t K, int64_t ldx,
+                                             const int32_t *row_token_dev, void *out_dev, int64_t ld_out,
+                                             int64_t M_out, void *stream)
+{
+    NVFP4_REQUIRE(T >= 0 && K >= 0 && M_out >= 0, NVFP4_ERR_INVALID_ARG, "moe_routed_rows_bf16: negative size");
+    if (M_out == 0 || K == 0) return NVFP4_OK;
+    NVFP4_REQUIRE(row_token_dev && out_dev && (T == 0 || x_dev), NVFP4_ERR_INVALID_ARG,
+                  "moe_routed_rows_bf16: null pointer");
+    NVFP4_REQUIRE(K % 8 == 0 && ldx >= K && ldx % 8 == 0 && ld_out >= K && ld_out % 8 == 0, NVFP4_ERR_ALIGNMENT,
+                  "moe_routed_rows_bf16: K, ldx and ld_out must be multiples of 8 with ldx, ld_out >= K");
+    NVFP4_REQUIRE((T == 0 || aligned16(x_dev)) && aligned16(out_dev), NVFP4_ERR_ALIGNMENT,
+                  "moe_routed_rows_bf16: pointers must be 16-byte aligned");
+    NVFP4_REQUIRE(M_out < (1ll << 31), NVFP4_ERR_UNSUPPORTED_SHAPE, "moe_routed_rows_bf16: too many rows");
+    dim3 grid((unsigned)M_out, (unsigned)((K + 2047) / 2048));
+    k_routed_rows_bf16<<<grid, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const uint4 *>(x_dev), T, K, ldx,
+                                                               row_token_dev, reinterpret_cast<uint4 *>(out_dev), ld_out);
+    return check_launch("k_routed_rows_bf16");
+}

@@ -35,18 +35,23 @@ def rac_channels(percent: float, K: int) -> int:
 
 class MoELayerW4A4:
     """rac_k: RAC channels of the gate/up input X (and of h unless rac_k_h is
-    given); see rac_channels for a percentage."""
+    given); see rac_channels for a percentage.  rac_scope "expert" selects the
+    channel sets per expert (nvfp4_quantize_experts): X through its complete
+    routed copy, h directly; rac_mode must then be "bf16"."""
 
     def __init__(self, w13: torch.Tensor, w2: torch.Tensor, tokens: int, topk: int, rac_k: int,
-                 seg_align: int = 256, rac_k_h: int | None = None, rac_mode: str = "bf16"):
+                 seg_align: int = 256, rac_k_h: int | None = None, rac_mode: str = "bf16",
+                 rac_scope: str = "tensor"):
         assert w13.dtype == torch.bfloat16 and w2.dtype == torch.bfloat16
         E, N13, H = w13.shape
         E2, H2, I = w2.shape
         assert E2 == E and H2 == H and N13 == 2 * I
         dev = w13.device
         self.E, self.H, self.I, self.T, self.k_r = E, H, I, tokens, topk
-        assert rac_mode in ("bf16", "nvfp4")
+        assert rac_mode in ("bf16", "nvfp4") and rac_scope in ("tensor", "expert")
+        assert rac_scope == "tensor" or (rac_mode == "bf16" and rac_k > 0 and (rac_k_h is None or rac_k_h > 0))
         self.rac_mode = rac_mode            # "nvfp4": second NVFP4 pass over the selected residual channels
+        self.rac_scope = rac_scope
         self.rac_k = rac_k
         self.rac_k_h = rac_k if rac_k_h is None else rac_k_h
         self.rac_ld = -(-rac_k // 64) * 64 if rac_k else 0
@@ -82,8 +87,19 @@ class MoELayerW4A4:
         self.ws_x = api._ws(lib.nvfp4_quantize_workspace_size(tokens, H), dev)
         self.ws_h = api._ws(lib.nvfp4_quantize_workspace_size(mp, I), dev)
         self.routing = None
+        if rac_scope == "expert":
+            # per-expert sets: [E x k] selections, the routed copy of X, and
+            # workspaces sized for the routed rows
+            self.xq.sel = torch.empty(E, rac_k, dtype=torch.int32, device=dev)
+            self.hq.sel = torch.empty(E, self.rac_k_h, dtype=torch.int32, device=dev)
+            self.xq.score = self.hq.score = None
+            self.x_routed = torch.empty(mp, H, dtype=torch.bfloat16, device=dev)
+            self.ws_x = api._ws(lib.nvfp4_quantize_experts_workspace_size(mp, H, E, seg_align), dev)
+            self.ws_h = api._ws(lib.nvfp4_quantize_experts_workspace_size(mp, I, E, seg_align), dev)
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor) -> torch.Tensor:
+        if self.rac_scope == "expert":
+            return self._forward_experts(x, logits)
         E, H, I, k, kh = self.E, self.H, self.I, self.rac_k, self.rac_k_h
         r = api.route(logits, self.k_r, self.m_pad, self.seg_align) if self.routing is None else self._route_into(logits)
         self.routing = r
@@ -109,6 +125,30 @@ class MoELayerW4A4:
         api.grouped_gemm(self.hq.codes, self.hq.scales, self.hq.s_t, self.m_pad, self.c2, self.sf2, self.s2,
                          H, I, E, r.offsets, seg_align=self.seg_align, rac_ld=self.rac_ld_h if kh else 0,
                          rho=self.hq.r_sel, w_sel=self.w_sel2,
+                         epilogue=api.EPI_SCATTER_ADD_F32, row_token=r.row_token, row_gate=r.row_gate, out=self.y)
+        return self.y
+
+    def _forward_experts(self, x: torch.Tensor, logits: torch.Tensor) -> torch.Tensor:
+        """The layer with one RAC channel set per expert for X and for h."""
+        E, H, I, k, kh, sa = self.E, self.H, self.I, self.rac_k, self.rac_k_h, self.seg_align
+        r = api.route(logits, self.k_r, self.m_pad, sa) if self.routing is None else self._route_into(logits)
+        self.routing = r
+        api.routed_rows_bf16(x, r.row_token, self.m_pad, out=self.x_routed)
+        api.quantize_experts(self.x_routed, r.offsets, E, sa, rac_k=k, rac_ld=self.rac_ld, out=self.xq,
+                             workspace=self.ws_x)
+        api.gather_weight_channels_cm_experts(self.c13_cm, self.sf13_cm, 2 * I, H, self.xq.sel, k, self.rac_ld,
+                                              out=self.w_sel13)
+        api.grouped_gemm(self.xq.codes, self.xq.scales, self.xq.s_t, self.m_pad, self.c13, self.sf13, self.s13,
+                         2 * I, H, E, r.offsets, seg_align=sa, rac_ld=self.rac_ld, rho=self.xq.r_sel,
+                         w_sel=self.w_sel13, epilogue=api.EPI_SWIGLU_BF16, row_token=r.row_token,
+                         row_gate=r.row_gate, out=self.h, amax_out=self.h_amax)
+        api.quantize_experts(self.h, r.offsets, E, sa, rac_k=kh, rac_ld=self.rac_ld_h, amax=self.h_amax,
+                             out=self.hq, workspace=self.ws_h)
+        api.gather_weight_channels_cm_experts(self.c2_cm, self.sf2_cm, H, I, self.hq.sel, kh, self.rac_ld_h,
+                                              out=self.w_sel2)
+        self.y.zero_()
+        api.grouped_gemm(self.hq.codes, self.hq.scales, self.hq.s_t, self.m_pad, self.c2, self.sf2, self.s2,
+                         H, I, E, r.offsets, seg_align=sa, rac_ld=self.rac_ld_h, rho=self.hq.r_sel, w_sel=self.w_sel2,
                          epilogue=api.EPI_SCATTER_ADD_F32, row_token=r.row_token, row_gate=r.row_gate, out=self.y)
         return self.y
 
