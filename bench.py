@@ -101,6 +101,7 @@ def parse():
     ap.add_argument("--no-w4a16", action="store_true", help="skip the trainer-side W4A16 line of the default run")
     ap.add_argument("--no-formats", action="store_true", help="skip the W4A4 / W8A8 / BF16 grouped-GEMM table")
     ap.add_argument("--no-sweep", action="store_true", help="skip the layer-error sweep over RAC channels and outliers")
+    ap.add_argument("--no-variants", action="store_true", help="skip the per-variant RAC step times")
     return ap.parse_args()
 
 
@@ -344,6 +345,14 @@ def run_ours(args):
         torch.cuda.empty_cache()
         out["gemm_formats"] = run_formats(args, dev)
         out["gpu_launches"] += out["gemm_formats"].pop("_launches")
+    if not args.no_variants:
+        # cost side of RAC: whole layer steps of the same workload without RAC
+        # and with each RAC variant
+        if "layer" in locals():
+            del layer
+        torch.cuda.empty_cache()
+        out["rac_variants"] = run_rac_variants(args, dev)
+        out["gpu_launches"] += out["rac_variants"].pop("_launches")
     if not args.no_sweep:
         # accuracy side of RAC: the error it leaves on one dense layer, by
         # compensated channel share and outlier strength (untimed)
@@ -354,6 +363,52 @@ def run_ours(args):
     if rank == 0:
         print(json.dumps(out), flush=True)
     return out
+
+
+def run_rac_variants(args, dev):
+    """Layer step time of the large layer without RAC and with each RAC
+    variant (same inputs and routing), CUDA events around whole steps."""
+    import torch
+    from quantization_nvfp4_quantize_b200 import workloads as wl
+    from quantization_nvfp4_quantize_b200 import moe as moe_mod
+    cfg = wl.CONFIGS[WORKLOAD]
+    x = wl.activations(cfg, args.seed, device=dev)
+    logits = wl.router_logits(cfg, args.seed, device=dev)
+    w13, w2 = wl.weights(cfg, args.seed, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    steps = max(3, min(args.steps, 5))
+    H, I = cfg.hidden, cfg.inter
+    variants = (
+        ("no_rac", dict(rac_k=0), 10),
+        ("rac_k128", dict(rac_k=cfg.rac_k), 16),
+        ("rac_50pct", dict(rac_k=moe_mod.rac_channels(50, H), rac_k_h=moe_mod.rac_channels(50, I)), 16),
+        ("rac_second_pass", dict(rac_k=cfg.rac_k, rac_mode="nvfp4"), 20),
+        ("rac_per_expert", dict(rac_k=cfg.rac_k, rac_scope="expert"), 17),
+    )
+    res, launches = {}, 0
+    for name, kw, n_launch in variants:
+        layer = moe_mod.MoELayerW4A4(w13, w2, cfg.tokens, cfg.topk, **kw)
+        for _ in range(2):
+            layer.forward(x, logits)
+        torch.cuda.synchronize()
+        s_ = torch.cuda.Event(enable_timing=True)
+        e_ = torch.cuda.Event(enable_timing=True)
+        s_.record(stream)
+        for _ in range(steps):
+            layer.forward(x, logits)
+        e_.record(stream)
+        torch.cuda.synchronize()
+        res[name] = {"ms_per_step": round(s_.elapsed_time(e_) / steps, 4)}
+        launches += n_launch * steps
+        del layer
+        torch.cuda.empty_cache()
+    base = res["no_rac"]["ms_per_step"]
+    for name in res:
+        res[name]["overhead_vs_no_rac"] = round(res[name]["ms_per_step"] / base - 1, 4)
+    res["k"] = {"rac_k128": [cfg.rac_k, cfg.rac_k], "rac_50pct": [moe_mod.rac_channels(50, H), moe_mod.rac_channels(50, I)]}
+    res["note"] = "whole layer steps of the bench workload (X side, h side), CUDA events around the steps"
+    res["_launches"] = launches
+    return res
 
 
 def run_error_sweep(args, dev):
