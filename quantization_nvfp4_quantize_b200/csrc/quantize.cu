@@ -708,7 +708,7 @@ __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__r
                                                               int64_t K, const int32_t *__restrict__ sel, int k,
                                                               int ld, __nv_bfloat16 *__restrict__ out, int sel_stride)
 {
-    extern __shared__ float gtile[];                   // [GCM_N features][cw channels of this chunk]
+    extern __shared__ __align__(16) uint16_t gtile[];  // bf16 [GCM_N features][cw channels of this chunk]
     __shared__ float e4[128];                          // E4M3 code -> value (weight scales are non-negative)
     __shared__ int32_t ssel[GCM_J];
     const int64_t e = blockIdx.y;
@@ -729,7 +729,7 @@ __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__r
     for (int idx = threadIdx.x; idx < cw * groups; idx += blockDim.x) {
         const int jj = idx % cw;
         const int f0 = (idx / cw) * 32;
-        float v[32];
+        uint16_t v[32];
         const int64_t ch = jj < kc ? (int64_t)ssel[jj] : -1;
         if (ch >= 0 && ch < K && n0 + f0 < N) {        // channels outside [0, K) give zeros
             const uint4 w = *reinterpret_cast<const uint4 *>(codes_cm + (e * K + ch) * (N / 2) + (n0 + f0) / 2);
@@ -744,12 +744,14 @@ __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__r
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int f = q * 8 + i;
-                    v[f] = __fmul_rn(c8[i], e4[(sw[f >> 2] >> (8 * (f & 3))) & 0x7Fu]);
+                    // e2m1 * sf has at most 6 significant bits: exact in bf16
+                    v[f] = __bfloat16_as_ushort(__float2bfloat16_rn(
+                        __fmul_rn(c8[i], e4[(sw[f >> 2] >> (8 * (f & 3))) & 0x7Fu])));
                 }
             }
         } else {
 #pragma unroll
-            for (int f = 0; f < 32; ++f) v[f] = 0.0f;
+            for (int f = 0; f < 32; ++f) v[f] = 0;
         }
 #pragma unroll
         for (int f = 0; f < 32; ++f) gtile[(f0 + f) * cw + jj] = v[f];
@@ -762,14 +764,8 @@ __global__ void __launch_bounds__(256) k_gather_w_channels_cm(const uint8_t *__r
         const int f = idx / cpr;
         const int jc = (idx - f * cpr) * 8;
         if (n0 + f >= N) break;                        // rows are monotone in idx
-        const float4 a = *reinterpret_cast<const float4 *>(gtile + f * cw + jc);
-        const float4 b = *reinterpret_cast<const float4 *>(gtile + f * cw + jc + 4);
-        uint4 o;
-        o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.x)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.y)) << 16);
-        o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.z)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.w)) << 16);
-        o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.x)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.y)) << 16);
-        o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.z)) | ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.w)) << 16);
-        *reinterpret_cast<uint4 *>(out + (e * N + n0 + f) * ld + j0 + jc) = o;
+        *reinterpret_cast<uint4 *>(out + (e * N + n0 + f) * ld + j0 + jc) =
+            *reinterpret_cast<const uint4 *>(gtile + f * cw + jc);
     }
 }
 
@@ -1191,7 +1187,7 @@ static nvfp4_status gather_cm(const uint8_t *codes_cm_dev, const uint8_t *scales
                   "nvfp4_gather_weight_channels_cm: need 0 <= k <= ld <= 16384, ld % 64 == 0");
     NVFP4_REQUIRE(aligned16(w_sel_dev) && aligned16(codes_cm_dev) && aligned16(scales_cm_dev), NVFP4_ERR_ALIGNMENT,
                   "nvfp4_gather_weight_channels_cm: pointers must be 16-byte aligned");
-    size_t smem = (size_t)std::min(ld, GCM_J) * GCM_N * sizeof(float);
+    size_t smem = (size_t)std::min(ld, GCM_J) * GCM_N * sizeof(uint16_t);
     {
         static std::once_flag once[64];
         static cudaError_t attr_err[64];
@@ -1200,7 +1196,7 @@ static nvfp4_status gather_cm(const uint8_t *codes_cm_dev, const uint8_t *scales
             return check_launch("nvfp4_gather_weight_channels_cm: device");
         std::call_once(once[dev], [&] {
             attr_err[dev] = cudaFuncSetAttribute(k_gather_w_channels_cm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)(GCM_J * GCM_N * sizeof(float)));
+                                                 (int)(GCM_J * GCM_N * sizeof(uint16_t)));
         });
         if (attr_err[dev] != cudaSuccess)
             return set_error(NVFP4_ERR_CUDA, "nvfp4_gather_weight_channels_cm: smem attribute: %s",
