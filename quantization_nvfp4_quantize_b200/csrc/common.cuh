@@ -183,12 +183,19 @@ __device__ __forceinline__ float2 recip_bracket(float den)
 
 // E4M3 code of the block scale fl(fl(a/6) / s_t), a >= 0; r6 = bracket of
 // 1/(6 s_t) (recip_bracket(fl(6 s_t)) encloses it: fl(6 s_t) is within 2^-24).
+// The division fallbacks are rare (arguments within ~2^-20 of a rounding
+// boundary) and kept out of line, so the streaming loops stay small.
+static __device__ __noinline__ uint32_t block_scale_code_div(float a, float s_t)
+{
+    return cvt_e4m3(__fdiv_rn(__fdiv_rn(a, 6.0f), s_t));
+}
+
 __device__ __forceinline__ uint32_t block_scale_code(float a, float s_t, float2 r6)
 {
     const uint32_t c2 = cvt_e4m3x2(__fmul_rn(a, r6.x), __fmul_rn(a, r6.y));
     const uint32_t c = c2 & 0xFFu;
     if ((c2 >> 8) == c) return c;
-    return cvt_e4m3(__fdiv_rn(__fdiv_rn(a, 6.0f), s_t));
+    return block_scale_code_div(a, s_t);
 }
 
 // Per E4M3 scale code, the per-tensor quantities of a block: its scale
@@ -243,6 +250,14 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w)
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
+// E2M1 codes of 8 elements by IEEE division (the out-of-line fallback).
+static __device__ __noinline__ uint32_t element_codes8_div(float2 v0, float2 v1, float2 v2, float2 v3, float d)
+{
+    const float y[8] = {__fdiv_rn(v0.x, d), __fdiv_rn(v0.y, d), __fdiv_rn(v1.x, d), __fdiv_rn(v1.y, d),
+                        __fdiv_rn(v2.x, d), __fdiv_rn(v2.y, d), __fdiv_rn(v3.x, d), __fdiv_rn(v3.y, d)};
+    return cvt_e2m1x8(y);
+}
+
 // E2M1 codes of 8 elements (one lane's half of a 16-block; 4 bytes, element
 // 2i in the low nibble of byte i) given the block's constants.
 __device__ __forceinline__ uint32_t element_codes8(const float2 v[4], const BlockConst &b)
@@ -257,13 +272,7 @@ __device__ __forceinline__ uint32_t element_codes8(const float2 v[4], const Bloc
     }
     const uint32_t wlo = cvt_e2m1x8(ylo);
     if (wlo == cvt_e2m1x8(yhi)) return wlo;
-    float y[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        y[2 * i] = __fdiv_rn(v[i].x, b.d);
-        y[2 * i + 1] = __fdiv_rn(v[i].y, b.d);
-    }
-    return cvt_e2m1x8(y);
+    return element_codes8_div(v[0], v[1], v[2], v[3], b.d);
 }
 
 // Dequantized values of 8 elements from their codes: pairs
@@ -294,12 +303,17 @@ __device__ __forceinline__ void residual8(const float2 v[4], const float2 xh[4],
     for (int i = 0; i < 4; ++i) R[i] = make_float2(__fsub_rn(v[i].x, xh[i].x), __fsub_rn(v[i].y, xh[i].y));
 }
 
+static __device__ __noinline__ uint32_t element_code1_div(float v, float d)
+{
+    return cvt_e2m1x2(__fdiv_rn(v, d), 0.0f) & 15u;
+}
+
 // Dequantized value fl(fl(e2m1(q) * sf) * s_t) of a single element.
 __device__ __forceinline__ float element_xhat1(float v, const BlockConst &b, float s_t)
 {
     const uint32_t c2 = cvt_e2m1x2(__fmul_rn(v, b.rlo), __fmul_rn(v, b.rhi));
     uint32_t q = c2 & 15u;
-    if ((c2 >> 4) != q) q = cvt_e2m1x2(__fdiv_rn(v, b.d), 0.0f) & 15u;
+    if ((c2 >> 4) != q) q = element_code1_div(v, b.d);
     const float sf = __low2float(*reinterpret_cast<const __half2 *>(&b.sf_h2));
     return __fmul_rn(__fmul_rn(e2m1x2_to_f32(q).x, sf), s_t);
 }

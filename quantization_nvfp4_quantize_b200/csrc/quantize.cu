@@ -268,7 +268,9 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
                 }
                 __syncwarp();
             }
-#pragma unroll
+            // the fan-out instance runs smaller as a rolled loop
+            constexpr int ROW_UNROLL = FAN ? 1 : QRPW;
+#pragma unroll ROW_UNROLL
             for (int i = 0; i < QRPW; ++i) {
                 const uint32_t r = rt + (uint32_t)(i * QWORKERS);
                 if (r >= r1) break;                                   // warp-uniform
