@@ -702,19 +702,13 @@ static nvfp4_status dispatch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, c
     const int64_t n_tiles = epilogue == MOE_EPI_SWIGLU_BF16 ? p.inter / 128 : p.N / BN;
     // Tile order: the scatter-add epilogue reduces into token rows that every
     // expert touches; grouping 2 n-tiles (512 output columns) keeps the band
-    // of output being reduced into small enough to stay in L2 while all
-    // experts' contributions to it arrive (16384 tokens x 4096 f32: 1114 us
-    // in plain order, 937 us in groups of 2).  NVFP4_GEMM_NGROUP overrides
-    // (must divide the n-tile count).
+    // of output being reduced into small (16384 tokens x 4096 f32: 1114 us in
+    // plain order, 937 us in groups of 2; groups of 1, 4 or 8 and a token-phase
+    // order of the m-tiles measured no better).
     int n_group = (int)n_tiles;
     if (epilogue == MOE_EPI_SCATTER_ADD_F32 && n_tiles % 2 == 0) n_group = 2;
-    if (const char *env = getenv("NVFP4_GEMM_NGROUP")) {
-        const int g = atoi(env);
-        if (g > 0 && n_tiles % g == 0) n_group = g;
-    }
     p.n_group = n_group;
     p.l2_hints = epilogue == MOE_EPI_SCATTER_ADD_F32 ? 1 : 0;
-    if (const char *env = getenv("NVFP4_GEMM_L2HINTS")) p.l2_hints = p.l2_hints && atoi(env) != 0;
     const int64_t max_tiles = (M_pad_max / seg_align) * n_tiles;
     const bool swiglu = epilogue == MOE_EPI_SWIGLU_BF16;
     if (pair) {
