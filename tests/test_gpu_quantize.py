@@ -421,3 +421,27 @@ def test_rac_second_pass_nvfp4_parity(cuda, M, K, k, ld):
     got = np_u16(q.r_sel)
     assert np.array_equal(got[:, :k], rho2)
     assert np.all(got[:, k:] == 0)
+
+
+def test_zero_row_chunks_match_oracle(cuda):
+    """Rows whose 256-channel chunks are all zero (the padding rows of routed
+    segments) take a short path in the kernel: +0 and -0 rows, rows zero in
+    only some chunks, and mixed rows give the oracle's codes (-0 -> code 8),
+    scale bytes, scores and QDQ values bit for bit."""
+    rng = np.random.default_rng(77)
+    M, K = 96, 1024
+    x = gen_x(rng, M, K)
+    x[0:8] = 0                                   # +0 rows
+    x[8:16] = 0x8000                             # -0 rows
+    x[16:24, :256] = 0                           # first chunk zero
+    x[24:32, 512:768] = 0x8000                   # a middle chunk of -0
+    x[32:40] = np.where(rng.random((8, K)) < 0.5, 0x8000, 0).astype(np.uint16)   # mixed signed zeros
+    x[40:48, 768:] = 0
+    x[40:48, 768] = 0x3F80                       # a single 1.0 in an otherwise zero chunk
+    _quant_parity(cuda, x, 16)
+    # QDQ (one tensor) over the same rows
+    w_qdq, s_t, codes, scales = api.qdq_weights(to_bf16_dev(x, cuda), want_packed=True)
+    torch.cuda.synchronize()
+    wq, s_ref, _ = oracle.qdq(x)
+    assert s_t.item() == np.float32(s_ref)
+    assert np.array_equal(np_u16(w_qdq), wq)
