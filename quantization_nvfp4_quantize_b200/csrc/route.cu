@@ -224,6 +224,21 @@ __global__ void __launch_bounds__(256) k_gather_rows_bf16(const uint4 *__restric
     }
 }
 
+// Every routed row r < M_out gets token row_token[r] of x, or zeros for a
+// padding row (row_token < 0): the copy is complete whatever the routing
+// left in the buffer before.
+__global__ void __launch_bounds__(256) k_routed_rows_bf16(const uint4 *__restrict__ x, int64_t T, int64_t K,
+                                                          int64_t ldx, const int32_t *__restrict__ row_token,
+                                                          uint4 *__restrict__ out, int64_t ld_out)
+{
+    const int64_t r = blockIdx.x;
+    const int64_t col = ((int64_t)blockIdx.y * 256 + threadIdx.x) * 8;
+    if (col >= K) return;
+    const int32_t t = row_token[r];
+    const uint4 v = (t >= 0 && t < T) ? x[((int64_t)t * ldx + col) >> 3] : make_uint4(0u, 0u, 0u, 0u);
+    out[(r * ld_out + col) >> 3] = v;
+}
+
 }  // namespace nvfp4
 
 using namespace nvfp4;
@@ -294,21 +309,6 @@ extern "C" nvfp4_status moe_route(const float *logits_dev, int64_t T, int32_t E,
     k_route_place<<<(unsigned)nblk, 1024, 0, st>>>(topk_idx_dev, topk_gate_dev, T, E, k_r, blkcnt, tot, seg_align,
                                                   offsets_dev, dst_row_dev, row_token_dev, row_gate_dev);
     return check_launch("k_route_place");
-}
-
-// Every routed row r < M_out gets token row_token[r] of x, or zeros for a
-// padding row (row_token < 0): the copy is complete whatever the routing
-// left in the buffer before.
-__global__ void __launch_bounds__(256) k_routed_rows_bf16(const uint4 *__restrict__ x, int64_t T, int64_t K,
-                                                          int64_t ldx, const int32_t *__restrict__ row_token,
-                                                          uint4 *__restrict__ out, int64_t ld_out)
-{
-    const int64_t r = blockIdx.x;
-    const int64_t col = ((int64_t)blockIdx.y * 256 + threadIdx.x) * 8;
-    if (col >= K) return;
-    const int32_t t = row_token[r];
-    const uint4 v = (t >= 0 && t < T) ? x[((int64_t)t * ldx + col) >> 3] : make_uint4(0u, 0u, 0u, 0u);
-    out[(r * ld_out + col) >> 3] = v;
 }
 
 extern "C" nvfp4_status moe_routed_rows_bf16(const void *x_dev, int64_t T, int64_t K, int64_t ldx,
