@@ -127,7 +127,10 @@ NVFP4_API int nvfp4_num_sms(void);
  *   rac_ld       row stride (elements) of r_sel, rac_ld >= rac_k,
  *                rac_ld % 64 == 0; columns [rac_k, rac_ld) are written as 0.
  *   sel_dev      int32 [rac_k]: selected channels, ascending.
- *   r_sel_dev    bf16 [M_out x rac_ld].
+ *   r_sel_dev    bf16 [M_out x rac_ld], or NULL: the channels are selected
+ *                but no residual is written (e.g. when
+ *                nvfp4_rac_residual_nvfp4 produces the RAC operand next;
+ *                rac_ld is then not checked).
  *   dev_status   optional int32 status word (see conventions).
  *   workspace    nvfp4_quantize_workspace_size(M, K) bytes, 16-byte aligned.
  * Only rows named as destinations are written; other output rows keep their

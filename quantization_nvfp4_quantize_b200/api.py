@@ -59,8 +59,10 @@ def quantize(x: torch.Tensor, *, rac_k: int = 0, rac_ld: int | None = None, s_t:
              amax: torch.Tensor | None = None,
              dst_rows: torch.Tensor | None = None, fanout: int = 1, m_out: int | None = None,
              m_valid: torch.Tensor | None = None, want_score: bool = False, out: Quantized | None = None,
-             workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None) -> Quantized:
-    """nvfp4_quantize on a bf16 [M, K] tensor (see the header for semantics)."""
+             workspace: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+             want_residual: bool = True) -> Quantized:
+    """nvfp4_quantize on a bf16 [M, K] tensor (see the header for semantics).
+    want_residual=False selects the RAC channels without writing r_sel."""
     lib = _lib.load()
     assert x.dtype == BF16 and x.dim() == 2 and x.stride(1) == 1
     M, K = x.shape
@@ -82,8 +84,8 @@ def quantize(x: torch.Tensor, *, rac_k: int = 0, rac_ld: int | None = None, s_t:
         workspace = _ws(lib.nvfp4_quantize_workspace_size(M, K), dev)
     check(lib.nvfp4_quantize(_p(x), M, K, x.stride(0), _p(m_valid), _p(s_t), _p(amax), _p(out.s_t), _p(dst_rows),
                              fanout, m_out, _p(out.codes), _p(out.scales), _p(out.score), rac_k, rac_ld,
-                             _p(out.sel), _p(out.r_sel), _p(dev_status), _p(workspace), workspace.numel(),
-                             _stream(dev)))
+                             _p(out.sel), _p(out.r_sel) if want_residual else None, _p(dev_status), _p(workspace),
+                             workspace.numel(), _stream(dev)))
     return out
 
 

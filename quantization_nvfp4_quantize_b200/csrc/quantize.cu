@@ -873,11 +873,12 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
                   "nvfp4_quantize: M_out must be >= M without dst_rows");
     NVFP4_REQUIRE(rac_k >= 0 && rac_k <= K, NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize: rac_k must be in [0, K]");
     if (rac_k > 0) {
-        NVFP4_REQUIRE(sel_dev && r_sel_dev, NVFP4_ERR_INVALID_ARG,
-                      "nvfp4_quantize: rac_k > 0 needs sel and r_sel");
-        NVFP4_REQUIRE(rac_ld >= rac_k && rac_ld % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
-                      "nvfp4_quantize: rac_ld must be >= rac_k and a multiple of 64");
-        NVFP4_REQUIRE(aligned16(r_sel_dev), NVFP4_ERR_ALIGNMENT, "nvfp4_quantize: r_sel must be 16-byte aligned");
+        NVFP4_REQUIRE(sel_dev, NVFP4_ERR_INVALID_ARG, "nvfp4_quantize: rac_k > 0 needs sel");
+        if (r_sel_dev) {
+            NVFP4_REQUIRE(rac_ld >= rac_k && rac_ld % 64 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+                          "nvfp4_quantize: rac_ld must be >= rac_k and a multiple of 64");
+            NVFP4_REQUIRE(aligned16(r_sel_dev), NVFP4_ERR_ALIGNMENT, "nvfp4_quantize: r_sel must be 16-byte aligned");
+        }
     }
     const bool want_score = score_dev != nullptr || rac_k > 0;
     size_t need = nvfp4_quantize_workspace_size(M, K);
@@ -938,7 +939,7 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
             return set_error(NVFP4_ERR_CUDA, "nvfp4_quantize: smem attribute: %s", cudaGetErrorString(attr_err[dev]));
         k_select_topk<<<1, 1024, smem, st>>>(score, (int)K, rac_k, sel_dev);
         if (check_launch("k_select_topk") != NVFP4_OK) return NVFP4_ERR_CUDA;
-        if (M > 0) {
+        if (M > 0 && r_sel_dev) {                         // no r_sel: the selection only
             const float *s_t_used = s_t_in_dev ? s_t_in_dev : s_t_out_dev;
             unsigned blocks = (unsigned)((M + 7) / 8);
             k_rac_residual<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, s_t_used,

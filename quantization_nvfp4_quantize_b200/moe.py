@@ -103,8 +103,9 @@ class MoELayerW4A4:
         E, H, I, k, kh = self.E, self.H, self.I, self.rac_k, self.rac_k_h
         r = api.route(logits, self.k_r, self.m_pad, self.seg_align) if self.routing is None else self._route_into(logits)
         self.routing = r
+        nvfp4_rac = self.rac_mode == "nvfp4"          # the second pass writes the RAC operand
         api.quantize(x, rac_k=k, rac_ld=self.rac_ld, dst_rows=r.dst_row, fanout=self.k_r, m_out=self.m_pad,
-                     out=self.xq, workspace=self.ws_x)
+                     out=self.xq, workspace=self.ws_x, want_residual=not nvfp4_rac)
         if k and self.rac_mode == "nvfp4":
             api.rac_residual_nvfp4(x, self.xq, k, self.rac_ld, dst_rows=r.dst_row, fanout=self.k_r, m_out=self.m_pad)
         if k:
@@ -115,7 +116,7 @@ class MoELayerW4A4:
                          w_sel=self.w_sel13, epilogue=api.EPI_SWIGLU_BF16, row_token=r.row_token,
                          row_gate=r.row_gate, out=self.h, amax_out=self.h_amax)
         api.quantize(self.h, rac_k=kh, rac_ld=self.rac_ld_h, m_out=self.m_pad, m_valid=r.offsets[E:],
-                     amax=self.h_amax, out=self.hq, workspace=self.ws_h)
+                     amax=self.h_amax, out=self.hq, workspace=self.ws_h, want_residual=not nvfp4_rac)
         if kh and self.rac_mode == "nvfp4":
             api.rac_residual_nvfp4(self.h, self.hq, kh, self.rac_ld_h, m_out=self.m_pad, m_valid=r.offsets[E:])
         if kh:

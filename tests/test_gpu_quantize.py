@@ -445,3 +445,20 @@ def test_zero_row_chunks_match_oracle(cuda):
     wq, s_ref, _ = oracle.qdq(x)
     assert s_t.item() == np.float32(s_ref)
     assert np.array_equal(np_u16(w_qdq), wq)
+
+
+def test_selection_without_residual(cuda):
+    """r_sel NULL with rac_k > 0: the channels are selected exactly as with a
+    residual output, and no residual is written."""
+    rng = np.random.default_rng(12)
+    M, K, k = 300, 1024, 40
+    x = gen_x(rng, M, K)
+    xd = to_bf16_dev(x, cuda)
+    full = api.quantize(xd, rac_k=k, want_score=True)
+    q = api.quantize(xd, rac_k=k, want_score=True, want_residual=False)
+    sentinel = torch.full_like(q.r_sel, 3.0)
+    q.r_sel.copy_(sentinel)
+    q = api.quantize(xd, rac_k=k, want_score=True, want_residual=False, out=q)
+    torch.cuda.synchronize()
+    assert torch.equal(q.sel, full.sel) and torch.equal(q.codes, full.codes)
+    assert torch.equal(q.r_sel, sentinel)
