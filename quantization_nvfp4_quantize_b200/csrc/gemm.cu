@@ -49,7 +49,8 @@
 // Tiles never span two experts (segments are multiples of the tile height);
 // the tile count comes from the device-side offsets (no host sync).  Tile
 // order: m-major, except that the scatter-add epilogue runs the n-tiles in
-// groups of 2, so the band of token rows being reduced into stays in L2.
+// groups of 2, so the band of output being reduced into is an eighth of Y
+// (much of it still leaves L2 between a row's contributions).
 //
 // Shared memory: a ring of stages (single 54 KB, pair 38 KB: 4 / 5 stages for
 // the bf16 epilogue, 3 / 5 for the f32 ones) plus, for the f32 epilogues, a
