@@ -178,6 +178,10 @@ __device__ __forceinline__ float tensor_scale_from_amax(float A)
 __device__ __forceinline__ float2 recip_bracket(float den)
 {
     const float r = __frcp_rn(den);
+    // 1/den above the binary32 range (den below 2^-128): the pair (0, inf)
+    // never encodes to one code for a non-zero argument, so every decision
+    // then takes the division
+    if (!(r < INFINITY)) return make_float2(0.0f, INFINITY);
     return make_float2(__fmul_rn(r, 1.0f - 0x1p-20f), __fmul_rn(r, 1.0f + 0x1p-20f));
 }
 

@@ -37,6 +37,10 @@ constexpr int QRPW = QROWS / QWORKERS;   // tile rows per worker warp
 constexpr uint32_t QPITCH = QCHUNK * 2;  // bytes per tile row
 constexpr uint32_t QTILE = QPITCH * QROWS;
 constexpr uint32_t QSMEM = QSTAGES * QTILE;   // 64 KB of tiles per CTA
+constexpr int MAX_EXPERTS = 256;      // expert sets of nvfp4_quantize_experts
+
+__device__ __forceinline__ __nv_bfloat162 bf162_bits(uint32_t w) { return *reinterpret_cast<__nv_bfloat162 *>(&w); }
+__device__ __forceinline__ __nv_bfloat16 bf16_from_bits(uint32_t w) { return __ushort_as_bfloat16((unsigned short)w); }
 
 // -------------------------------------------------------------------- amax
 
@@ -509,10 +513,234 @@ __global__ void __launch_bounds__(1024) k_select_topk(const double *__restrict__
 
 // --------------------------------------------------------- RAC residual
 
-// One warp per input row; lane j handles selected channel S_j.  The block of
-// S_j is re-quantized from x with the same arithmetic as k_quantize (one lane
+// Block constants of the E4M3 scale codes 0..127 (every code a non-negative
+// block scale takes) for tensor scale s_t, filled by the CTA's first 128
+// threads; the caller synchronizes before reading.
+__device__ __forceinline__ void fill_block_table(float4 *tab, float s_t)
+{
+    if (threadIdx.x < 128) {
+        const BlockConst b = block_const(threadIdx.x, s_t);
+        tab[threadIdx.x] = make_float4(b.d, b.rlo, b.rhi, __uint_as_float(b.sf_h2));
+    }
+}
+
+// E4M3 scale code of a 16-block given as its two 16-byte halves, with the
+// arithmetic of k_quantize.  The block max is taken on bf16 pairs
+// (max.bf16x2 ignores a NaN operand, as fmaxf does).
+__device__ __forceinline__ uint32_t block_code16(uint4 u0, uint4 u1, float s_t, float2 r6)
+{
+    const uint32_t mk = 0x7FFF7FFFu;
+    const __nv_bfloat162 m2 = __hmax2(
+        __hmax2(__hmax2(bf162_bits(u0.x & mk), bf162_bits(u0.y & mk)), __hmax2(bf162_bits(u0.z & mk), bf162_bits(u0.w & mk))),
+        __hmax2(__hmax2(bf162_bits(u1.x & mk), bf162_bits(u1.y & mk)), __hmax2(bf162_bits(u1.z & mk), bf162_bits(u1.w & mk))));
+    const uint32_t mb = *reinterpret_cast<const uint32_t *>(&m2);
+    return block_scale_code(fmaxf(bf16lo(mb), bf16hi(mb)), s_t, r6);
+}
+
+static __device__ __noinline__ uint32_t rho_bf16_div(float R, float s_t)
+{
+    const __nv_bfloat16 h = __float2bfloat16_rn(__fdiv_rn(R, s_t));
+    return *reinterpret_cast<const uint16_t *>(&h);
+}
+
+// bf16(fl(R / s_t)) as a 16-bit pattern; rs = recip_bracket(s_t).  Both
+// roundings are monotone, so when the bracketing products round to the same
+// bf16 that is the value of the division (else the division is evaluated).
+__device__ __forceinline__ uint32_t rho_bf16(float R, float s_t, float2 rs)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(R, rs.x), __fmul_rn(R, rs.y));
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(&h);
+    if ((w & 0xFFFFu) == (w >> 16)) return w & 0xFFFFu;
+    return rho_bf16_div(R, s_t);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// E2M1 codes of (lo, hi) in bits 0..3 / 4..7.
+__device__ __forceinline__ uint32_t e2m1x2_bits(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// R = fl(x - xhat) of one element of a block with constants b: the code of
+// fl(x / d) from the bracketing products (the division when they differ),
+// xhat = fl(fl(e2m1 * sf) * s_t) with the e2m1 * sf product exact in f16.
+__device__ __forceinline__ float element_residual(float xv, const BlockConst &b, float s_t)
+{
+    uint32_t c = e2m1x2_bits(__fmul_rn(xv, b.rlo), __fmul_rn(xv, b.rhi));
+    if ((c >> 4) != (c & 15u)) {
+        const uint32_t q = element_code1_div(xv, b.d);
+        c = q * 0x11u;
+    }
+    uint32_t h2;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.u8.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t"
+        "mul.rn.f16x2 %0, %0, %2;\n\t}"
+        : "=r"(h2) : "r"(c), "r"(b.sf_h2));
+    const float qsf = __low2float(*reinterpret_cast<const __half2 *>(&h2));
+    return __fsub_rn(xv, __fmul_rn(qsf, s_t));
+}
+
+constexpr int RC_WARPS = 8;            // warps per CTA, each streaming its own rows
+constexpr int RC_CHUNK = 2048;         // channels of a row staged at a time (4 KB)
+constexpr int RC_GROUPS = 8;           // 4-column output groups a lane holds: windows of 1024 columns
+constexpr int RC_WIN = RC_GROUPS * 128;
+
+// Dynamic shared memory of k_rac_residual: two row pieces per warp.
+static size_t rac_residual_smem(int64_t K)
+{
+    return (size_t)RC_WARPS * 2 * (size_t)std::min<int64_t>(K, RC_CHUNK) * 2;
+}
+
+// rho[dst, j] = bf16(R[r, S_j] / s_t) for every valid row r and each of its
+// destination rows.  The selected channels cover most 32-byte sectors of a
+// row, so rows are streamed whole: each warp owns a sequence of rows, taken
+// in pieces of up to 2048 channels, and copies the next piece into shared
+// memory (cp.async, 16 bytes a lane) while it works on the current one.  Per
+// piece the warp first takes the scale codes of all of the piece's 16-blocks
+// (k_quantize's arithmetic, so R matches the quantized tensor bit for bit);
+// then lane l handles the output columns 4 l .. 4 l + 3 of every 128, for the
+// selected channels that fall in the piece, keeping a window of 1024 columns
+// in registers until the row's last piece and storing them as 8-byte words
+// (a row with more columns passes over its pieces once per window).
+// Per-expert sets: row r uses the set of expert e with
+// offsets[e] <= r < offsets[e + 1].  Columns [k, ld) are written as zeros.
+__global__ void __launch_bounds__(RC_WARPS * 32) k_rac_residual(
+    const __nv_bfloat16 *__restrict__ x, int64_t ldx, int64_t M, int64_t K,
+    const int32_t *__restrict__ m_valid, const float *__restrict__ s_t_ptr,
+    const int32_t *__restrict__ sel, int k, int ld,
+    const int32_t *__restrict__ dst_rows, int fanout, int64_t M_out, __nv_bfloat16 *__restrict__ r_sel,
+    const int32_t *__restrict__ expert_offsets, int E)
+{
+    extern __shared__ __align__(16) uint8_t rsm[];               // [RC_WARPS][2][piece]
+    __shared__ float4 tab[128];
+    __shared__ uint8_t bcode[RC_WARPS][RC_CHUNK / 16];
+    __shared__ int32_t offs[MAX_EXPERTS + 1];
+    const float s_t = *s_t_ptr;
+    fill_block_table(tab, s_t);
+    if (expert_offsets)
+        for (int i = threadIdx.x; i <= E; i += blockDim.x) offs[i] = expert_offsets[i];
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int64_t Me = M;
+    if (m_valid) Me = min(Me, (int64_t)max(*m_valid, 0));
+    const float2 r6 = recip_bracket(__fmul_rn(6.0f, s_t));
+    const float2 rs = recip_bracket(s_t);
+    const int piece = (int)min(K, (int64_t)RC_CHUNK);
+    const int npiece = (int)((K + piece - 1) / piece);
+    const int nwin = (ld + RC_WIN - 1) / RC_WIN;
+    const int64_t nw = (int64_t)gridDim.x * RC_WARPS;
+    uint8_t *wbuf = rsm + (size_t)warp * 2 * piece * 2;
+    uint8_t *codes = bcode[warp];
+
+    // a warp's units in order: rows gw, gw + nw, ...; per row its windows,
+    // per window its pieces
+    auto issue = [&](int64_t r, int p, int s) {
+        if (r < Me) {
+            const int c0 = p * piece;
+            const int nv = (int)min((int64_t)piece, K - c0) / 8;      // 16-byte vectors of the piece
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(x + r * ldx + c0);
+            const uint32_t dst = ptx::smem_u32(wbuf + s * piece * 2);
+            for (int v = lane; v < nv; v += 32) cp_async16(dst + v * 16, src + v * 16);
+        }
+        cp_async_commit();                           // possibly empty: one group per unit keeps the count
+    };
+
+    int64_t r = (int64_t)blockIdx.x * RC_WARPS + warp;
+    int win = 0, p = 0;
+    int64_t rn = r;
+    int winn = 0, pn = 0;
+    uint2 acc[RC_GROUPS];
+    issue(r, p, 0);
+    for (int s = 0; r < Me; s ^= 1) {
+        if (++pn == npiece) {
+            pn = 0;
+            if (++winn == nwin) { winn = 0; rn += nw; }
+        }
+        issue(rn, pn, s ^ 1);
+        cp_async_wait1();                            // this lane's copies of the unit have landed
+        __syncwarp();                                // ... and every lane's
+        const int c0 = p * piece;
+        const int w = (int)min((int64_t)piece, K - c0);
+        const __nv_bfloat16 *row = reinterpret_cast<const __nv_bfloat16 *>(wbuf + s * piece * 2);
+        for (int bi = lane; bi < w / 16; bi += 32) {
+            const uint4 *bp = reinterpret_cast<const uint4 *>(row + bi * 16);
+            codes[bi] = (uint8_t)block_code16(bp[0], bp[1], s_t, r6);
+        }
+        __syncwarp();
+        const int32_t *srow = sel;
+        if (expert_offsets) {
+            int lo = 0, hi = E;
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (offs[mid] <= r) lo = mid; else hi = mid;
+            }
+            srow += (int64_t)lo * k;
+        }
+        if (p == 0) {
+#pragma unroll
+            for (int g = 0; g < RC_GROUPS; ++g) acc[g] = make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int g = 0; g < RC_GROUPS; ++g) {
+            const int j0 = win * RC_WIN + g * 128 + lane * 4;
+            if (win * RC_WIN + g * 128 >= ld) break;     // warp-uniform
+            if (j0 < ld && j0 < k) {                     // a group lies wholly inside or outside [0, ld)
+                uint32_t o[4] = {acc[g].x & 0xFFFFu, acc[g].x >> 16, acc[g].y & 0xFFFFu, acc[g].y >> 16};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    if (j0 + t < k) {
+                        const int ch = srow[j0 + t] - c0;
+                        if (ch >= 0 && ch < w) {
+                            const float4 bt = tab[codes[ch >> 4]];
+                            const BlockConst b{bt.x, bt.y, bt.z, __float_as_uint(bt.w)};
+                            o[t] = rho_bf16(element_residual(__bfloat162float(row[ch]), b, s_t), s_t, rs);
+                        }
+                    }
+                }
+                acc[g] = make_uint2(o[0] | (o[1] << 16), o[2] | (o[3] << 16));
+            }
+        }
+        if (p == npiece - 1) {                          // the window is complete: store it
+            const int32_t *drow = dst_rows ? dst_rows + r * fanout : nullptr;
+            const int nd = drow ? fanout : 1;
+            for (int d = 0; d < nd; ++d) {
+                const int64_t dst = drow ? (int64_t)drow[d] : r;
+                if (dst < 0 || dst >= M_out) continue;
+                uint2 *out = reinterpret_cast<uint2 *>(r_sel + dst * ld);
+#pragma unroll
+                for (int g = 0; g < RC_GROUPS; ++g) {
+                    const int j0 = win * RC_WIN + g * 128 + lane * 4;
+                    if (win * RC_WIN + g * 128 >= ld) break;
+                    if (j0 < ld) out[j0 >> 2] = acc[g];
+                }
+            }
+        }
+        __syncwarp();                                // the piece is read: its buffer may be refilled
+        r = rn;
+        win = winn;
+        p = pn;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// The same rho for a selection that touches few of a row's blocks: one warp
+// per input row, lane j handles selected channel S_j and loads only S_j's
+// 32-byte block, re-quantized with the arithmetic of k_quantize (one lane
 // takes the whole 16-block max), giving the residual bit for bit.
-__global__ void __launch_bounds__(256) k_rac_residual(
+__global__ void __launch_bounds__(256) k_rac_residual_sparse(
     const __nv_bfloat16 *__restrict__ x, int64_t ldx, int64_t M, int64_t K,
     const int32_t *__restrict__ m_valid, const float *__restrict__ s_t_ptr,
     const int32_t *__restrict__ sel, int k, int ld,
@@ -559,6 +787,42 @@ __global__ void __launch_bounds__(256) k_rac_residual(
             if (dst >= 0 && dst < M_out) r_sel[dst * ld + j] = outv;
         }
     }
+}
+
+// Launch of the RAC residual: the streaming kernel (one wave of resident
+// CTAs, fewer for small M) when the selected channels are at least as many as
+// a row's 16-blocks, else the per-channel kernel.
+static nvfp4_status launch_rac_residual(const __nv_bfloat16 *x, int64_t ldx, int64_t M, int64_t K,
+                                        const int32_t *m_valid, const float *s_t, const int32_t *sel, int k, int ld,
+                                        const int32_t *dst_rows, int fanout, int64_t M_out, __nv_bfloat16 *r_sel,
+                                        const int32_t *expert_offsets, int E, cudaStream_t st)
+{
+    if ((int64_t)k * 16 < K) {
+        // fewer selected channels than blocks: most of a row's sectors are not needed
+        k_rac_residual_sparse<<<(unsigned)((M + 7) / 8), 256, 0, st>>>(x, ldx, M, K, m_valid, s_t, sel, k, ld, dst_rows,
+                                                                     fanout, M_out, r_sel, expert_offsets, E);
+        return check_launch("k_rac_residual_sparse");
+    }
+    const size_t smem = rac_residual_smem(K);
+    static std::once_flag once[64];
+    static cudaError_t attr_err[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return set_error(NVFP4_ERR_CUDA, "k_rac_residual: no device");
+    std::call_once(once[dev], [&] {
+        attr_err[dev] = cudaFuncSetAttribute(k_rac_residual, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)rac_residual_smem(RC_CHUNK));
+    });
+    if (attr_err[dev] != cudaSuccess)
+        return set_error(NVFP4_ERR_CUDA, "k_rac_residual: smem attribute: %s", cudaGetErrorString(attr_err[dev]));
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_rac_residual, RC_WARPS * 32, smem) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const unsigned blocks = (unsigned)std::max<int64_t>(
+        1, std::min<int64_t>((M + RC_WARPS - 1) / RC_WARPS, (int64_t)num_sms() * per_sm));
+    k_rac_residual<<<blocks, RC_WARPS * 32, smem, st>>>(x, ldx, M, K, m_valid, s_t, sel, k, ld, dst_rows, fanout,
+                                                        M_out, r_sel, expert_offsets, E);
+    return check_launch("k_rac_residual");
 }
 
 // ----------------------------------------- RAC second-pass (NVFP4) variant
@@ -941,12 +1205,10 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
         if (check_launch("k_select_topk") != NVFP4_OK) return NVFP4_ERR_CUDA;
         if (M > 0 && r_sel_dev) {                         // no r_sel: the selection only
             const float *s_t_used = s_t_in_dev ? s_t_in_dev : s_t_out_dev;
-            unsigned blocks = (unsigned)((M + 7) / 8);
-            k_rac_residual<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, s_t_used,
-                                                   sel_dev, rac_k, rac_ld, dst_rows_dev,
-                                                   dst_rows_dev ? fanout : 1, M_out, (__nv_bfloat16 *)r_sel_dev,
-                                                   nullptr, 0);
-            if (check_launch("k_rac_residual") != NVFP4_OK) return NVFP4_ERR_CUDA;
+            if (launch_rac_residual((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, s_t_used, sel_dev, rac_k,
+                                    rac_ld, dst_rows_dev, dst_rows_dev ? fanout : 1, M_out,
+                                    (__nv_bfloat16 *)r_sel_dev, nullptr, 0, st) != NVFP4_OK)
+                return NVFP4_ERR_CUDA;
         }
     }
     return NVFP4_OK;
@@ -1044,10 +1306,9 @@ extern "C" nvfp4_status nvfp4_quantize_experts(const void *x_dev, int64_t M, int
     if (check_launch("k_select_topk") != NVFP4_OK) return NVFP4_ERR_CUDA;
     if (M > 0) {
         const float *s_t_used = s_t_in_dev ? s_t_in_dev : s_t_out_dev;
-        k_rac_residual<<<(unsigned)((M + 7) / 8), 256, 0, st>>>((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev,
-                                                               s_t_used, sel_dev, rac_k, rac_ld, nullptr, 1, M,
-                                                               (__nv_bfloat16 *)r_sel_dev, offsets_dev, E);
-        if (check_launch("k_rac_residual") != NVFP4_OK) return NVFP4_ERR_CUDA;
+        if (launch_rac_residual((const __nv_bfloat16 *)x_dev, ldx, M, K, m_valid_dev, s_t_used, sel_dev, rac_k, rac_ld,
+                                nullptr, 1, M, (__nv_bfloat16 *)r_sel_dev, offsets_dev, E, st) != NVFP4_OK)
+            return NVFP4_ERR_CUDA;
     }
     return NVFP4_OK;
 }

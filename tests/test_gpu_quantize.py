@@ -91,6 +91,31 @@ def test_quantize_zero_and_tiny(cuda):
     _quant_parity(cuda, y, 16)
 
 
+def test_quantize_reciprocal_overflow(cuda):
+    """A tensor scale and block scales below 2^-128, whose reciprocals overflow
+    binary32: every decision there must come from the division.  Codes, scale
+    bytes, s_t and rho are bit-exact; scores are not compared (their binary32
+    partial sums of R^2 underflow at this magnitude)."""
+    rng = np.random.default_rng(11)
+    x = gen_x(rng, 200, 512, scale=1e-37)
+    x[:, 32:40] = 0
+    x[5, :] = 0
+    x[:, 64:96] = gen_x(rng, 200, 32, outliers=0, scale=1e-39)
+    x[::3, 64:72] = 0
+    ref = oracle.quantize(x)
+    d = oracle.e4m3_decode(ref.sf.astype(np.uint8)).astype(np.float32) * np.float32(ref.s_t)
+    assert np.float32(ref.s_t) < 2.0 ** -128 and np.sum((d > 0) & (d < 2.0 ** -128)) > 0
+    k = 24
+    q = api.quantize(to_bf16_dev(x, cuda), rac_k=k, want_score=True)
+    torch.cuda.synchronize()
+    assert q.s_t.item() == np.float32(ref.s_t)
+    assert np.array_equal(q.codes.cpu().numpy(), ref.codes)
+    assert np.array_equal(unswizzle(q.scales, 200, 512), ref.sf)
+    sel = q.sel.cpu().numpy()[:k]
+    assert len(set(sel.tolist())) == k and sel.min() >= 0 and sel.max() < 512
+    assert np.array_equal(np_u16(q.r_sel)[:, :k], oracle.rac_residual(ref.resid, ref.s_t, sel))
+
+
 def test_quantize_empty(cuda):
     x = torch.empty(0, 256, dtype=torch.bfloat16, device=cuda)
     q = api.quantize(x, rac_k=0, m_out=0, want_score=True)
@@ -98,8 +123,11 @@ def test_quantize_empty(cuda):
     assert q.s_t.item() == 1.0 and np.all(q.score.cpu().numpy() == 0)
 
 
-def test_quantize_fanout_and_valid_rows(cuda):
-    """dst_rows fan-out writes every copy; m_valid limits the rows read."""
+@pytest.mark.parametrize("k", [16, 48])
+def test_quantize_fanout_and_valid_rows(cuda, k):
+    """dst_rows fan-out writes every copy; m_valid limits the rows read.  With
+    k = 16 the selection touches few of a row's 32 blocks (residuals from the
+    selected blocks only); with k = 48 rows are streamed whole."""
     rng = np.random.default_rng(6)
     M, K, F = 200, 512, 3
     x = gen_x(rng, M, K)
@@ -107,15 +135,15 @@ def test_quantize_fanout_and_valid_rows(cuda):
     perm[7, 1] = -1
     m_out = -(-(M * F + 100) // 128) * 128
     xd = to_bf16_dev(x, cuda)
-    q = api.quantize(xd, rac_k=16, dst_rows=torch.from_numpy(perm).to(cuda), fanout=F, m_out=m_out)
+    q = api.quantize(xd, rac_k=k, dst_rows=torch.from_numpy(perm).to(cuda), fanout=F, m_out=m_out)
     torch.cuda.synchronize()
     ref = oracle.quantize(x)
     codes = q.codes.cpu().numpy()
     sf = unswizzle(q.scales, m_out, K)
     rsel = np_u16(q.r_sel)
     score = oracle.channel_score(ref.resid)
-    sel = q.sel.cpu().numpy()[:16]
-    check_selection(sel, score, oracle.select_topk(score, 16), 16)
+    sel = q.sel.cpu().numpy()[:k]
+    check_selection(sel, score, oracle.select_topk(score, k), k)
     rho = oracle.rac_residual(ref.resid, ref.s_t, sel)
     for r in range(M):
         for j in range(F):
@@ -124,10 +152,10 @@ def test_quantize_fanout_and_valid_rows(cuda):
                 continue
             assert np.array_equal(codes[d], ref.codes[r])
             assert np.array_equal(sf[d], ref.sf[r])
-            assert np.array_equal(rsel[d, :16], rho[r])
+            assert np.array_equal(rsel[d, :k], rho[r])
     # m_valid: only the first 77 rows count
     mv = torch.tensor([77], dtype=torch.int32, device=cuda)
-    q2 = api.quantize(xd, rac_k=16, m_valid=mv, want_score=True)
+    q2 = api.quantize(xd, rac_k=k, m_valid=mv, want_score=True)
     torch.cuda.synchronize()
     ref2 = oracle.quantize(x[:77])
     assert q2.s_t.item() == np.float32(ref2.s_t)
@@ -370,10 +398,12 @@ def test_near_boundary_sweep_matches_oracle(cuda):
         assert np.array_equal(q.codes.cpu().numpy(), codes[g])
 
 
-@pytest.mark.parametrize("M,K,k", [(300, 2048, 1024), (129, 768, 768), (64, 4096, 2048)])
+@pytest.mark.parametrize("M,K,k", [(300, 2048, 1024), (129, 768, 768), (64, 4096, 2048), (200, 4096, 300),
+                                   (40, 16384, 1100)])
 def test_quantize_rac_percent_channels(cuda, M, K, k):
-    """RAC on "the top k% of channels" (50% and 100%): selection, scores and
-    residual operand bit-exact beyond the former 256-channel cap."""
+    """RAC on "the top k% of channels" (7% to 100%, rows staged in one or
+    several pieces and column windows): selection, scores and residual operand
+    bit-exact beyond the former 256-channel cap."""
     rng = np.random.default_rng(M + K + k)
     _quant_parity(cuda, gen_x(rng, M, K), k)
 
