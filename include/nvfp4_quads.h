@@ -264,7 +264,9 @@ NVFP4_API nvfp4_status nvfp4_qdq_weights(const void *w_dev, int64_t G, int64_t r
  * moe_route -- top-k_r expert routing of T tokens over E experts and the
  * expert-grouped routed-row layout used by the grouped GEMMs.
  *
- *   logits_dev   float32 [T x E], E <= 256, 1 <= k_r <= min(E, 8).
+ *   logits_dev   float32 [T x E], E <= 256, 1 <= k_r <= min(E, 8); -0 ranks
+ *                as +0, and a NaN logit (not a routing input) would rank
+ *                above every number.
  *   topk_idx_dev int32 [T x k_r]: experts by descending logit (equal logits:
  *                lower expert first).
  *   topk_gate_dev float32 [T x k_r]: softmax over the k_r selected logits.

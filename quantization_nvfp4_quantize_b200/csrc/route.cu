@@ -1,8 +1,10 @@
 // route.cu -- MoE top-k routing and the expert-grouped routed-row layout.
 //
 //   k_route_topk   one warp per token, 32 tokens per CTA ("routing block"):
-//                  k_r rounds of warp argmax over the E logits (equal logits:
-//                  lower expert), softmax over the selected logits; the
+//                  k_r rounds of warp argmax over the E logits (warp max of
+//                  order-preserving keys, then warp min of the experts holding
+//                  it: equal logits go to the lower expert), softmax over the
+//                  selected logits; the
 //                  block's per-expert counts in shared memory -> blkcnt.
 //   k_route_scan   one warp per expert: an exclusive scan of its counts over
 //                  the routing blocks, and the expert's total.
@@ -37,13 +39,18 @@ __global__ void __launch_bounds__(1024) k_route_topk(const float *__restrict__ l
         const int64_t t = (int64_t)blockIdx.x * RB + tt;
         if (t >= T) break;                                    // warp-uniform
         const int nslots = (E + 31) >> 5;                    // populated 32-expert slots
-        float l[MAX_EXPERTS / 32];
+        // order-preserving keys of the logits (-0 taken as +0, so equal
+        // logits have equal keys); 0 marks an empty slot
+        uint32_t key[MAX_EXPERTS / 32];
 #pragma unroll
         for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-            int e = lane + 32 * i;
-            l[i] = (i < nslots && e < E) ? logits[t * E + e] : -INFINITY;
+            const int e = lane + 32 * i;
+            key[i] = 0u;
+            if (i < nslots && e < E) {
+                const uint32_t u = __float_as_uint(logits[t * E + e] + 0.0f);
+                key[i] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+            }
         }
-        unsigned taken = 0;      // bit i: expert lane + 32 i already selected
         float sel_l[MAX_TOPK];   // fully unrolled below: stays in registers
         int sel_e[MAX_TOPK];
 #pragma unroll
@@ -51,25 +58,21 @@ __global__ void __launch_bounds__(1024) k_route_topk(const float *__restrict__ l
             sel_l[j] = -INFINITY;
             sel_e[j] = 0;
             if (j < kr) {
-                float bv = -INFINITY;
-                int be = 0x7fffffff;
+                // the largest remaining key, then the lowest expert holding it
+                uint32_t lm = 0u;
 #pragma unroll
-                for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-                    if (i >= nslots) break;
-                    int e = lane + 32 * i;
-                    if (e < E && !((taken >> i) & 1u)) {
-                        if (be == 0x7fffffff || l[i] > bv) { bv = l[i]; be = e; }
-                    }
-                }
+                for (int i = 0; i < MAX_EXPERTS / 32; ++i) lm = max(lm, key[i]);
+                const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
+                uint32_t le = 0xffffffffu;
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
-                }
-                sel_l[j] = bv;
+                for (int i = MAX_EXPERTS / 32 - 1; i >= 0; --i)
+                    if (key[i] == m) le = (uint32_t)(lane + 32 * i);
+                const int be = (int)__reduce_min_sync(0xffffffffu, le);
                 sel_e[j] = be;
-                if ((be & 31) == lane) taken |= 1u << (be >> 5);
+                sel_l[j] = __uint_as_float((m & 0x80000000u) ? (m & 0x7FFFFFFFu) : ~m);
+#pragma unroll
+                for (int i = 0; i < MAX_EXPERTS / 32; ++i)
+                    if (be == lane + 32 * i) key[i] = 0u;         // taken
             }
         }
         // softmax over the selected logits: lane j < k_r handles slot j; z is
