@@ -366,14 +366,29 @@ __global__ void __launch_bounds__(QTHREADS, QCTAS_PER_SM) k_quantize(const __gri
 
 // ----------------------------------------------------------- score reduce
 
-__global__ void k_score_reduce(const double *__restrict__ partials, int64_t P, int64_t K,
-                               double *__restrict__ score)
+// score[c] = sum over the P row-range partials of channel c.  A CTA takes 32
+// channels (one per lane); its 8 warps sum interleaved eighths of the
+// partials (warp w: q = w, w + 8, ...), then warp 0 adds the 8 sums in warp
+// order: a fixed order, so the scores are deterministic.
+constexpr int SR_WARPS = 8;
+
+__global__ void __launch_bounds__(SR_WARPS * 32) k_score_reduce(const double *__restrict__ partials, int64_t P,
+                                                               int64_t K, double *__restrict__ score)
 {
-    int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= K) return;
+    __shared__ double part[SR_WARPS][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t c = (int64_t)blockIdx.x * 32 + lane;
     double s = 0.0;
-    for (int64_t q = 0; q < P; ++q) s += partials[q * K + c];
-    score[c] = s;
+    if (c < K)
+        for (int64_t q = warp; q < P; q += SR_WARPS) s += partials[q * K + c];
+    part[warp][lane] = s;
+    __syncthreads();
+    if (warp == 0 && c < K) {
+        double t = part[0][lane];
+#pragma unroll
+        for (int w = 1; w < SR_WARPS; ++w) t += part[w][lane];
+        score[c] = t;
+    }
 }
 
 // Per-expert scores from row-group partials: row group q covers rows
@@ -1187,7 +1202,7 @@ extern "C" nvfp4_status nvfp4_quantize(const void *x_dev, int64_t M, int64_t K, 
     if (launch_quantize(want_score, x_dev, M, workspace, p, grid, st) != NVFP4_OK) return NVFP4_ERR_CUDA;
 
     if (want_score) {
-        k_score_reduce<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(partials, P, K, score);
+        k_score_reduce<<<(unsigned)((K + 31) / 32), SR_WARPS * 32, 0, st>>>(partials, P, K, score);
         if (check_launch("k_score_reduce") != NVFP4_OK) return NVFP4_ERR_CUDA;
     }
     if (rac_k > 0) {
