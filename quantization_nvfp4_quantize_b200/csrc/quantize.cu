@@ -438,16 +438,19 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *smem_warp, int &
 }
 
 // One CTA of 1024 threads.  Scores are non-negative binary64, whose bit
-// patterns order like their values; an 8-pass MSB-first radix select finds
-// the k-th largest key, then channels are taken in ascending index order:
-// every key above it, and the lowest-index keys equal to it.
+// patterns order like their values; an MSB-first radix select over 8-bit
+// digits finds the k-th largest key (stopping early once a single key holds
+// the selected prefix: that key is the k-th), then channels are taken in
+// ascending index order: every key above it, and the lowest-index keys equal
+// to it.
 __global__ void __launch_bounds__(1024) k_select_topk(const double *__restrict__ score, int K, int k,
                                                       int32_t *__restrict__ sel)
 {
     extern __shared__ unsigned long long keys[];
     __shared__ unsigned int hist[256];
     __shared__ int scan_tmp[33];
-    __shared__ int s_digit, s_rem;
+    __shared__ int s_digit, s_rem, s_cnt;
+    __shared__ unsigned long long s_key;
     const int tid = threadIdx.x;
     if (k <= 0) return;
     score += (int64_t)blockIdx.x * K;                 // one score vector (and set) per block
@@ -488,11 +491,20 @@ __global__ void __launch_bounds__(1024) k_select_topk(const double *__restrict__
                 }
                 s_digit = 255 - 8 * tid - b;
                 s_rem = rem - (int)a;
+                s_cnt = (int)cnt[b];
             }
         }
         __syncthreads();
         prefix |= (unsigned long long)s_digit << shift;
         mask |= 0xFFull << shift;
+        if (s_cnt == 1 && shift > 0) {
+            // one key holds the prefix: it is the k-th largest (s_rem == 1)
+            for (int i = tid; i < K; i += blockDim.x)
+                if ((keys[i] & mask) == prefix) s_key = keys[i];
+            __syncthreads();
+            prefix = s_key;
+            break;
+        }
     }
     const unsigned long long kth = prefix;
     const int take_eq = s_rem;          // keys equal to kth to take, lowest index first
