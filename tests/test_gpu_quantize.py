@@ -163,6 +163,33 @@ def test_quantize_fanout_and_valid_rows(cuda, k):
     np.testing.assert_allclose(q2.score.cpu().numpy(), oracle.channel_score(ref2.resid), rtol=SCORE_RTOL)
 
 
+def test_fanout_residual_pieces_and_windows(cuda):
+    """Residuals streamed in two row pieces (K = 4096) and two column windows
+    (ld = 1152), written to three routed rows each, some of them skipped."""
+    rng = np.random.default_rng(12)
+    M, K, F, k = 96, 4096, 3, 1100
+    x = gen_x(rng, M, K, outliers=40)
+    perm = rng.permutation(M * F + 50)[: M * F].astype(np.int32).reshape(M, F)
+    perm[4, 2] = -1
+    perm[9, 0] = M * F + 10_000          # beyond m_out: skipped
+    m_out = M * F + 50
+    q = api.quantize(to_bf16_dev(x, cuda), rac_k=k, rac_ld=1152, dst_rows=torch.from_numpy(perm).to(cuda),
+                     fanout=F, m_out=m_out)
+    torch.cuda.synchronize()
+    ref = oracle.quantize(x)
+    sel = q.sel.cpu().numpy()[:k]
+    score = oracle.channel_score(ref.resid)
+    check_selection(sel, score, oracle.select_topk(score, k), k)
+    rho = oracle.rac_residual(ref.resid, ref.s_t, sel)
+    rsel = np_u16(q.r_sel)
+    for r in range(M):
+        for j in range(F):
+            d = perm[r, j]
+            if 0 <= d < m_out:
+                assert np.array_equal(rsel[d, :k], rho[r]), (r, j)
+                assert np.all(rsel[d, k:] == 0)
+
+
 def test_select_ties(cuda):
     """Equal channel scores: lower channel index first (all-equal columns)."""
     x = np.tile(gen_x(np.random.default_rng(7), 1, 64), (50, 4))     # K = 256, repeated column groups
